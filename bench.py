@@ -1,0 +1,346 @@
+"""Benchmark: MXFP4 attention forward (UOS + PNQ) on the video-DiT-shaped workload.
+
+One step = one full pass of the hot path through the library's public C-ABI call
+mxattn_forward: quantize Q and K along d and V along keys (three quantizer launches), then the
+fused tcgen05 attention kernel, on B=1, H=40, N=32760, d=128, non-causal, seeded synthetic
+inputs resident in HBM. Inputs (3 x 335 MB of bf16) exceed the 126 MB L2, so no flush is needed.
+
+Multi-GPU (torchrun): every rank runs its own independent problem of the same shape (weak
+scaling, no data-path collective); the step time is the max over ranks.
+
+--impl reference runs the CPU oracle (numpy fp64) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "video_dit"
+METRIC = "MXFP4 attention fwd TFLOP/s (video-DiT 1x40x32760x128, UOS+PNQ)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+FP4_PER_BF16 = 4.0          # nominal dense ratio: 9 PFLOP/s fp4 vs 2.25 PFLOP/s bf16
+ATTN_SOURCES = ["mxfp4_microscaled_bit_quantize_b200/csrc/attn_fwd_sm100.cu",
+                "mxfp4_microscaled_bit_quantize_b200/csrc/sm100_ptx.cuh"]
+QUANT_SOURCES = ["mxfp4_microscaled_bit_quantize_b200/csrc/quantize.cu",
+                 "mxfp4_microscaled_bit_quantize_b200/csrc/sm100_ptx.cuh"]
+
+
+def sources_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def profile_traffic(name: str, src_hash: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != src_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(cfg, rows: int, head: int = 0):
+    """CPU oracle on a bounded sample: quantize one head's Q/K/V, then `rows` query rows of it."""
+    from mxfp4_microscaled_bit_quantize_b200 import synthetic
+    from oracle import attention as oa
+    from oracle import mxfp4 as mx
+
+    q = synthetic.head_bf16(cfg, "q", 0, head).double().numpy()
+    g = head * cfg.Hkv // cfg.Hq
+    k = synthetic.head_bf16(cfg, "k", 0, g).double().numpy()
+    v = synthetic.head_bf16(cfg, "v", 0, g).double().numpy()
+    t0 = time.perf_counter()
+    (qd, kd, vd), _ = oa.dequantized_qkv(q[:rows], k, v, mx.SCALE_UOS)
+    idx = np.arange(rows)
+    oa.attention_rows(qd, idx, kd, vd, causal=cfg.causal, mode=mx.SCALE_UOS, pnq=True)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * rows * cfg.N * cfg.d / (2.0 if cfg.causal else 1.0)
+    return flops, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def run_reference(args, rank: int) -> None:
+    from mxfp4_microscaled_bit_quantize_b200 import synthetic
+    if rank != 0:
+        return
+    cfg = synthetic.ATTN_CONFIGS[WORKLOAD]
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(cfg, rows)
+    flops = secs = 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(cfg, rows)
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    sample = (f"{rows} query rows of head 0 (Q/K/V of that head quantized, then online-softmax attention "
+              f"over all {cfg.N} keys) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, **cfg.describe(), "scale_mode": "UOS",
+                                            "pnq": True, "sample_rows": rows},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    from mxfp4_microscaled_bit_quantize_b200 import api, build, synthetic
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synthetic.ATTN_CONFIGS[WORKLOAD]
+    B, Hq, Hkv, N, d = cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.d
+    q, k, v = synthetic.attn_inputs(cfg)
+    q_h, k_h, v_h = (t.pin_memory() for t in (q, k, v))
+    dq, dk, dv = (t.to(dev) for t in (q_h, k_h, v_h))
+    ws = api.alloc_workspace(B, Hq, Hkv, N, d, dev)
+    out = torch.empty((B, Hq, N, d), dtype=torch.float32, device=dev)
+    out_h = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def step():
+        api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_UOS, ws)
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, True, ws)
+
+    for _ in range(args.warmup):
+        step()
+    if api.mxattn_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout during warm-up")
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_UOS, ws)
+            ev[i][1].record(stream)
+            api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, True, ws)
+            ev[i][2].record(stream)
+        stop.record(stream)
+        barrier()
+    if api.mxattn_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout in the timed region")
+    total_ms = start.elapsed_time(stop)
+    quant_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+
+    # end to end through the public call with host buffers: H2D inputs, forward, D2H output
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = out.numel() * out.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(q_h, non_blocking=True)
+        dk.copy_(k_h, non_blocking=True)
+        dv.copy_(v_h, non_blocking=True)
+        api.mxattn_forward(dq, dk, dv, causal=cfg.causal, scale_mode=api.SCALE_UOS, pnq=True, workspace=ws,
+                           out=out)
+        out_h.copy_(out, non_blocking=True)
+    e_stop.record(stream)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_stop) / e2e_steps
+
+    # standalone quantizer on its own workload (65536 x 1024 bf16), two buffer sets > L2
+    xq = [synthetic.quant_input().to(dev) for _ in range(2)]
+    qbuf = [api.mxattn_quantize(x, False, api.SCALE_UOS) for x in xq]
+    for i in range(5):
+        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
+    barrier()
+    qs, qe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    qiters = 50
+    qs.record(stream)
+    for i in range(qiters):
+        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
+    qe.record(stream)
+    barrier()
+    quant_alone_ms = qs.elapsed_time(qe) / qiters
+    del qbuf
+
+    # max over ranks
+    vals = torch.tensor([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms = (float(x) for x in vals.tolist())
+    if rank != 0:
+        return
+
+    flops = cfg.flops
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    elems = B * Hq * N * d + 2 * B * Hkv * N * d
+    # algorithmic bytes of the three quantizer launches: bf16 in, packed codes + scales out
+    quant_bytes = elems * 2 + elems // 2 + elems // 32
+    qa_elems = xq[0].numel()
+    qa_bytes = qa_elems * 2 + qa_elems // 2 + qa_elems // 32
+    line = {
+        "metric": METRIC,
+        "value": world * flops / (step_ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1xe2m1->f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, **cfg.describe(), "scale_mode": "UOS", "pnq": True,
+                   "out_dtype": "f32", "l2": "inputs 3x335 MB bf16 > 126 MB L2, no flush",
+                   "parallelism": f"independent problem per GPU x{world}"},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / fp4_peak, "kernel": "mxattn_fwd_kernel<128>",
+                     "peak_note": f"{peaks['source']} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16 ratio)",
+                     "traffic": profile_traffic("attn_fwd_video_dit.json", sources_hash(ATTN_SOURCES)),
+                     "algorithmic_flops_per_launch": flops, "ms_per_launch": attn_ms},
+        "quantizer": {"in_step_gbs": quant_bytes / (quant_ms * 1e-3) / 1e9, "in_step_ms": quant_ms,
+                      "standalone_65536x1024_gbs": qa_bytes / (quant_alone_ms * 1e-3) / 1e9,
+                      "standalone_ms": quant_alone_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
+                      "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        f, dt = oracle_sample(cfg, args.cpu_rows)
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{args.cpu_rows} query rows of head 0 (that head's Q/K/V "
+                                          f"quantized, attention over all {cfg.N} keys), {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=128)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,141 @@
+/*
+ * mxattn.h -- C ABI of the MXFP4 attention library for NVIDIA B200 (sm_100a).
+ *
+ * What it computes
+ * ----------------
+ * MXFP4 (OCP Microscaling) block quantization and MXFP4 attention forward as the MXAttention
+ * paper defines it ("MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+ * Quantization for MXFP4 Attention", abstract):
+ *   - 32-element blocks of E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; "Quantization
+ *     Error" page, section "Where the error comes from") sharing one E8M0 power-of-two scale;
+ *     values are rounded to nearest-even on the grid and saturate at 6.
+ *   - Scale exponent of a block with max magnitude amax:
+ *       MXATTN_SCALE_OCP: e = floor(log2 amax) - 2        (the OCP MX v1.0 rule)
+ *       MXATTN_SCALE_UOS: smallest e with amax / 2^e <= 7.25 (Universal Optimal Scaling)
+ *     An all-zero block gets scale byte 0 and all-zero codes.
+ *   - Attention: Q, K quantized along the head dimension, V along keys; S = Q K^T as a
+ *     block-scaled FP4 contraction; FlashAttention online softmax over 128-key tiles in
+ *     increasing key order (running max, history rescale, fp32 accumulation, final
+ *     normalisation; "EFQ-Softmax" abstract). With pnq = 1 (Pre-Normalization Quantization)
+ *     the unnormalised exponentials P~ = exp(S/sqrt(d) - m) are quantized to MXFP4 along keys
+ *     before the row sum, and that same dequantized operand feeds both P~V and the row sum.
+ *     With pnq = 0 the row sum uses the unquantized fp32 P~ (exp-then-quantize baseline).
+ *     Softmax scale is fixed at 1/sqrt(d).
+ *
+ * Conventions
+ * -----------
+ *   - Every pointer argument named as device memory must be a CUDA device pointer on the
+ *     current device. The caller owns every buffer; the library never allocates device memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are asynchronous on it.
+ *   - Argument errors are detected on the host and returned before anything is launched.
+ *     Launch errors return MXATTN_ERR_CUDA. A device-side pipeline timeout (every wait inside
+ *     the kernels is bounded) is recorded in the workspace and reported by
+ *     mxattn_check_status().
+ *   - Inputs must be finite; NaN / Inf inputs give unspecified codes.
+ *   - Packed E2M1 layout: two codes per byte, element 2i in bits 0..3, element 2i+1 in bits
+ *     4..7; code = sign << 3 | magnitude index. E8M0 byte = e + 127 (never 0xFF).
+ */
+#ifndef MXATTN_H_
+#define MXATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1 } mxattn_scale_mode;
+
+typedef enum { MXATTN_OUT_F32 = 0, MXATTN_OUT_BF16 = 1 } mxattn_out_dtype;
+
+typedef enum {
+  MXATTN_OK = 0,
+  MXATTN_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, negative or inconsistent size   */
+  MXATTN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not in {64, 128})        */
+  MXATTN_ERR_WORKSPACE = 3,    /* workspace smaller than mxattn_forward_workspace_size()      */
+  MXATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call or a kernel launch failed      */
+  MXATTN_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait (reported by check_status)*/
+} mxattn_status;
+
+/*
+ * mxattn_quantize -- MXFP4-quantize `batch` bf16 matrices of shape [rows, cols] (row-major,
+ * contiguous, device memory; `x` 2-byte aligned, 16-byte alignment enables vector loads).
+ * (Method: "Quantization Error" page, "Where the error comes from"; MXAttention abstract, UOS.)
+ *
+ *   transpose = 0: blocks of 32 along cols.  codes  [batch][rows][ceil(cols/32) * 16] (uint8)
+ *                                            scales [batch][rows][ceil(cols/32)]      (uint8)
+ *   transpose = 1: blocks of 32 along rows (e.g. V along keys), written transposed:
+ *                                            codes  [batch][cols][ceil(rows/32) * 16]
+ *                                            scales [batch][cols][ceil(rows/32)]
+ * A partial last block is zero-padded (padding never raises amax and encodes as +0).
+ * `codes` must be 16-byte aligned. Sizes must satisfy batch*rows*ceil(cols/32) < 2^31 and,
+ * for transpose = 1, batch <= 65535. Empty inputs (any size 0) are a no-op returning MXATTN_OK.
+ */
+mxattn_status mxattn_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int transpose,
+                              int scale_mode, uint8_t* codes, uint8_t* scales, void* stream);
+
+/*
+ * Bytes of device workspace mxattn_forward needs: quantized Q, K, V^T in the tensor-core
+ * layouts plus a 256-byte status area. 0 for invalid shapes.
+ */
+size_t mxattn_forward_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * mxattn_forward -- MXFP4 attention forward (MXAttention abstract: UOS + PNQ; OCP baseline).
+ *   q   : bf16 [B, Hq,  N, d] contiguous, device, 16-byte aligned
+ *   k, v: bf16 [B, Hkv, N, d] contiguous, device, 16-byte aligned
+ *   out : [B, Hq, N, d] fp32 (out_dtype = MXATTN_OUT_F32) or bf16, device, 16-byte aligned
+ *   Query head h reads KV head h / (Hq / Hkv) (contiguous GQA groups); Hq % Hkv == 0.
+ *   causal = 1 masks keys after the query position. scale_mode applies to Q, K, V and P~.
+ *   Supported: d in {64, 128}, 1 <= N, B*Hq*ceil(N/128) < 2^31.
+ *   workspace: device memory of at least mxattn_forward_workspace_size(...) bytes, 256-byte
+ *   aligned; its contents on entry are ignored; it must not be used concurrently by another
+ *   call. The call runs the quantizer three times (Q, K, V^T) and then the fused kernel.
+ */
+mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                             int N, int d, int causal, int scale_mode, int pnq, int out_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The two halves of mxattn_forward, for callers that time or reuse them separately:
+ *   mxattn_forward_prepare quantizes q, k, v into the workspace;
+ *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same
+ *   shapes and scale_mode as the prepare call).
+ */
+mxattn_status mxattn_forward_prepare(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                                     int N, int d, int scale_mode, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+mxattn_status mxattn_forward_attend(void* out, int B, int Hq, int Hkv, int N, int d, int causal,
+                                    int scale_mode, int pnq, int out_dtype, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
+ * mxattn_forward_debug -- mxattn_forward that also dumps the quantized P~ operand of query
+ * rows [r0, r1) of head dbg_bh (= b * Hq + h): p_codes [r1-r0][Npad/2] packed codes and
+ * p_scales [r1-r0][Npad/32] scale bytes in absolute key order, Npad = ceil(N/128)*128
+ * (device memory). Meant for parity tests on small shapes.
+ */
+mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                   int Hkv, int N, int d, int causal, int scale_mode, int pnq, int out_dtype,
+                                   void* workspace, size_t workspace_bytes, void* stream, int dbg_bh,
+                                   int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales);
+
+/*
+ * mxattn_check_status -- synchronises `stream`, reads and clears the workspace status word.
+ * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last check (the
+ * raw code goes to *detail when detail != NULL), MXATTN_ERR_CUDA on a CUDA error, else MXATTN_OK.
+ */
+mxattn_status mxattn_check_status(void* workspace, void* stream, unsigned int* detail);
+
+/* Static string for a status code. */
+const char* mxattn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int mxattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXATTN_H_ */

@@ -1,0 +1,154 @@
+"""Torch-facing wrappers of the C ABI: they only check tensors, allocate outputs with torch and
+marshal pointers, sizes and the current CUDA stream. Every step of the computation runs in the
+library's kernels; there is no CPU path."""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+
+SCALE_OCP, SCALE_UOS = 0, 1
+OUT_F32, OUT_BF16 = 0, 1
+KV_TILE = 128
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def npad(N: int) -> int:
+    return -(-N // KV_TILE) * KV_TILE
+
+
+def mxattn_quantize(x: torch.Tensor, transpose: bool = False, scale_mode: int = SCALE_UOS):
+    """MXFP4-quantize the last two axes [rows, cols] of a bf16 CUDA tensor.
+
+    transpose=False: blocks of 32 along cols -> codes [..., rows, ceil(cols/32)*16], scales [..., rows, ceil(cols/32)].
+    transpose=True:  blocks of 32 along rows -> codes [..., cols, ceil(rows/32)*16], scales [..., cols, ceil(rows/32)].
+    """
+    _need(x, "x")
+    if x.dim() < 2:
+        raise ValueError("x must have at least 2 dimensions")
+    lead = tuple(x.shape[:-2])
+    rows, cols = int(x.shape[-2]), int(x.shape[-1])
+    batch = math.prod(lead) if lead else 1
+    if transpose:
+        nb = -(-rows // 32)
+        codes = torch.empty(lead + (cols, nb * 16), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lead + (cols, nb), dtype=torch.uint8, device=x.device)
+    else:
+        nb = -(-cols // 32)
+        codes = torch.empty(lead + (rows, nb * 16), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lead + (rows, nb), dtype=torch.uint8, device=x.device)
+    lib = _lib.load()
+    st = lib.mxattn_quantize(x.data_ptr(), batch, rows, cols, int(bool(transpose)), int(scale_mode),
+                             codes.data_ptr(), scales.data_ptr(), _stream(x.device))
+    _lib.check(st, "mxattn_quantize")
+    return codes, scales
+
+
+def workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib.load().mxattn_forward_workspace_size(B, Hq, Hkv, N, d))
+
+
+def alloc_workspace(B: int, Hq: int, Hkv: int, N: int, d: int, device) -> torch.Tensor:
+    n = workspace_size(B, Hq, Hkv, N, d)
+    if n == 0:
+        raise ValueError("unsupported attention shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _shapes(q, k, v):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+        if t.dim() != 4:
+            raise ValueError(f"{n} must be [B, H, N, d]")
+    B, Hq, N, d = (int(s) for s in q.shape)
+    if tuple(k.shape) != tuple(v.shape) or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    return B, Hq, int(k.shape[1]), N, d
+
+
+def _out(q, out_dtype, out):
+    dt = torch.float32 if out_dtype in (OUT_F32, torch.float32) else torch.bfloat16
+    if out is None:
+        out = torch.empty(q.shape, dtype=dt, device=q.device)
+    else:
+        _need(out, "out", dt)
+    return out, (OUT_F32 if dt == torch.float32 else OUT_BF16)
+
+
+def mxattn_forward(q, k, v, causal: bool = False, scale_mode: int = SCALE_UOS, pnq: bool = True,
+                   out_dtype=torch.float32, workspace: torch.Tensor | None = None,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """MXFP4 attention forward (UOS / OCP scaling, PNQ on / off). q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16."""
+    B, Hq, Hkv, N, d = _shapes(q, k, v)
+    out, od = _out(q, out_dtype, out)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, N, d, q.device)
+    lib = _lib.load()
+    st = lib.mxattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                            int(bool(causal)), int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                            workspace.numel(), _stream(q.device))
+    _lib.check(st, "mxattn_forward")
+    return out
+
+
+def mxattn_forward_prepare(q, k, v, scale_mode: int, workspace: torch.Tensor) -> None:
+    B, Hq, Hkv, N, d = _shapes(q, k, v)
+    st = _lib.load().mxattn_forward_prepare(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d,
+                                            int(scale_mode), workspace.data_ptr(), workspace.numel(),
+                                            _stream(q.device))
+    _lib.check(st, "mxattn_forward_prepare")
+
+
+def mxattn_forward_attend(out: torch.Tensor, B: int, Hq: int, Hkv: int, N: int, d: int, causal: bool,
+                          scale_mode: int, pnq: bool, workspace: torch.Tensor) -> torch.Tensor:
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    st = _lib.load().mxattn_forward_attend(out.data_ptr(), B, Hq, Hkv, N, d, int(bool(causal)),
+                                           int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                                           workspace.numel(), _stream(out.device))
+    _lib.check(st, "mxattn_forward_attend")
+    return out
+
+
+def mxattn_forward_debug(q, k, v, dbg_bh: int, r0: int, r1: int, causal: bool = False,
+                         scale_mode: int = SCALE_UOS, pnq: bool = True, out_dtype=torch.float32,
+                         workspace: torch.Tensor | None = None):
+    """mxattn_forward plus the quantized P~ of rows [r0, r1) of head dbg_bh (= b*Hq + h):
+    returns (out, p_codes [r1-r0, Npad/2], p_scales [r1-r0, Npad/32])."""
+    B, Hq, Hkv, N, d = _shapes(q, k, v)
+    out, od = _out(q, out_dtype, None)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, N, d, q.device)
+    npd = npad(N)
+    pc = torch.zeros((r1 - r0, npd // 2), dtype=torch.uint8, device=q.device)
+    ps = torch.zeros((r1 - r0, npd // 32), dtype=torch.uint8, device=q.device)
+    st = _lib.load().mxattn_forward_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
+                                          Hkv, N, d, int(bool(causal)), int(scale_mode), int(bool(pnq)), od,
+                                          workspace.data_ptr(), workspace.numel(), _stream(q.device),
+                                          dbg_bh, r0, r1, pc.data_ptr(), ps.data_ptr())
+    _lib.check(st, "mxattn_forward_debug")
+    return out, pc, ps
+
+
+def mxattn_check_status(workspace: torch.Tensor) -> int:
+    """Synchronises the current stream; returns the device status word (0 = ok)."""
+    detail = ctypes.c_uint(0)
+    st = _lib.load().mxattn_check_status(workspace.data_ptr(), _stream(workspace.device),
+                                         ctypes.byref(detail))
+    if st not in (0, 5):
+        _lib.check(st, "mxattn_check_status")
+    return int(detail.value)

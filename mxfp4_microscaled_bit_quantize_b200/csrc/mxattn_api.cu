@@ -1,0 +1,314 @@
+// Host side of the C ABI declared in include/mxattn.h: argument checks, workspace carving,
+// TMA tensor-map encoding and kernel launches. No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mxattn.h"
+#include "mxattn_internal.h"
+
+using namespace mxattn;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr int kTile = 128;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t qc, qs, kc, ks, vc, vs, total;
+  int npad;
+};
+
+// status word at offset 0; every region 1 KiB aligned (TMA needs 16 B, bulk copies 16 B).
+bool ws_layout(int B, int Hq, int Hkv, int N, int d, WsLayout* L) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || (d != 64 && d != 128) || Hq % Hkv != 0) return false;
+  const size_t npad = align_up(static_cast<size_t>(N), kTile);
+  const size_t tiles = npad / kTile;
+  if (static_cast<uint64_t>(B) * Hq * tiles >= (1ull << 31)) return false;
+  if (static_cast<uint64_t>(B) * Hq * npad >= (1ull << 31)) return false;
+  size_t off = kAlign;  // status area
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L->qc = take(static_cast<size_t>(B) * Hq * npad * (d / 2));
+  L->qs = take(static_cast<size_t>(B) * Hq * tiles * 512);
+  L->kc = take(static_cast<size_t>(B) * Hkv * npad * (d / 2));
+  L->ks = take(static_cast<size_t>(B) * Hkv * tiles * 512);
+  L->vc = take(static_cast<size_t>(B) * Hkv * d * (npad / 2));
+  L->vs = take(static_cast<size_t>(B) * Hkv * tiles * 512);
+  L->total = off;
+  L->npad = static_cast<int>(npad);
+  return true;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }();
+  return fn;
+}
+
+// 2-D uint8 tensor map over a row-major [rows, row_bytes] byte matrix, box [box_rows, box_bytes].
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_bytes,
+              uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_bytes, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
+                           int scale_mode, void* ws, size_t ws_bytes, cudaStream_t st, const WsLayout& L) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (d < kTile) {
+    // scale atoms have room for 128 rows / 4 blocks; d = 64 leaves part of them unused
+    if (cudaMemsetAsync(w + L.qs, 0, L.kc - L.qs, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    if (cudaMemsetAsync(w + L.ks, 0, L.vc - L.ks, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    if (cudaMemsetAsync(w + L.vs, 0, L.total - L.vs, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  }
+  RowQuantParams rq{};
+  rq.x = static_cast<const __nv_bfloat16*>(q);
+  rq.heads = static_cast<uint32_t>(B * Hq);
+  rq.rows = static_cast<uint32_t>(N);
+  rq.rows_pad = static_cast<uint32_t>(L.npad);
+  rq.cols = static_cast<uint32_t>(d);
+  rq.kb = static_cast<uint32_t>(d / 32);
+  rq.codes = w + L.qc;
+  rq.scales = w + L.qs;
+  rq.mode = scale_mode;
+  rq.sf_layout = kSfAtom;
+  rq.vec_ok = aligned(q, 16) ? 1 : 0;
+  if (launch_quantize_rows(rq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  rq.x = static_cast<const __nv_bfloat16*>(k);
+  rq.heads = static_cast<uint32_t>(B * Hkv);
+  rq.codes = w + L.kc;
+  rq.scales = w + L.ks;
+  rq.vec_ok = aligned(k, 16) ? 1 : 0;
+  if (launch_quantize_rows(rq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  ColQuantParams cq{};
+  cq.x = static_cast<const __nv_bfloat16*>(v);
+  cq.heads = static_cast<uint32_t>(B * Hkv);
+  cq.rows = static_cast<uint32_t>(N);
+  cq.cols = static_cast<uint32_t>(d);
+  cq.nblk = static_cast<uint32_t>(L.npad / 32);
+  cq.codes = w + L.vc;
+  cq.scales = w + L.vs;
+  cq.mode = scale_mode;
+  cq.sf_layout = kSfAtom;
+  cq.vec_ok = aligned(v, 16) ? 1 : 0;
+  if (launch_quantize_cols(cq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  (void)ws_bytes;
+  return MXATTN_OK;
+}
+
+mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int causal, int scale_mode, int pnq,
+                          int out_dtype, void* ws, cudaStream_t st, const WsLayout& L, int dbg_bh, int dbg_r0,
+                          int dbg_r1, uint8_t* p_codes, uint8_t* p_scales) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle qk_swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_map(&tq, w + L.qc, d / 2, static_cast<uint64_t>(B) * Hq * L.npad, d / 2, kTile, qk_swz) ||
+      !make_map(&tk, w + L.kc, d / 2, static_cast<uint64_t>(B) * Hkv * L.npad, d / 2, kTile, qk_swz) ||
+      !make_map(&tv, w + L.vc, L.npad / 2, static_cast<uint64_t>(B) * Hkv * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
+    return MXATTN_ERR_CUDA;
+  AttnParams p{};
+  p.qsf = w + L.qs;
+  p.ksf = w + L.ks;
+  p.vsf = w + L.vs;
+  p.out = out;
+  p.out_bf16 = (out_dtype == MXATTN_OUT_BF16) ? 1 : 0;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.Npad = L.npad;
+  p.causal = causal ? 1 : 0;
+  p.mode = scale_mode;
+  p.pnq = pnq ? 1 : 0;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  p.status = reinterpret_cast<unsigned int*>(w);
+  p.dbg_codes = p_codes;
+  p.dbg_scales = p_scales;
+  p.dbg_bh = dbg_bh;
+  p.dbg_r0 = dbg_r0;
+  p.dbg_r1 = dbg_r1;
+  return launch_attention(tq, tk, tv, p, d, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+mxattn_status check_forward_args(const void* q, const void* k, const void* v, const void* out, int B, int Hq,
+                                 int Hkv, int N, int d, int scale_mode, int out_dtype, const void* ws,
+                                 size_t ws_bytes, WsLayout* L) {
+  if (scale_mode != MXATTN_SCALE_OCP && scale_mode != MXATTN_SCALE_UOS) return MXATTN_ERR_INVALID_ARG;
+  if (out_dtype != MXATTN_OUT_F32 && out_dtype != MXATTN_OUT_BF16) return MXATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return MXATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
+  if (!ws_layout(B, Hq, Hkv, N, d, L)) return MXATTN_ERR_UNSUPPORTED;
+  if (q && !aligned(q, 16)) return MXATTN_ERR_INVALID_ARG;
+  if (k && !aligned(k, 16)) return MXATTN_ERR_INVALID_ARG;
+  if (v && !aligned(v, 16)) return MXATTN_ERR_INVALID_ARG;
+  if (out && !aligned(out, 16)) return MXATTN_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return MXATTN_ERR_INVALID_ARG;
+  if (ws_bytes < L->total) return MXATTN_ERR_WORKSPACE;
+  return MXATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mxattn_version(void) { return 100; }
+
+const char* mxattn_status_string(int status) {
+  switch (status) {
+    case MXATTN_OK: return "ok";
+    case MXATTN_ERR_INVALID_ARG: return "invalid argument";
+    case MXATTN_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case MXATTN_ERR_WORKSPACE: return "workspace too small";
+    case MXATTN_ERR_CUDA: return "CUDA error";
+    case MXATTN_ERR_TIMEOUT: return "device pipeline timeout";
+    default: return "unknown status";
+  }
+}
+
+mxattn_status mxattn_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int transpose,
+                              int scale_mode, uint8_t* codes, uint8_t* scales, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return MXATTN_ERR_INVALID_ARG;
+  if (scale_mode != MXATTN_SCALE_OCP && scale_mode != MXATTN_SCALE_UOS) return MXATTN_ERR_INVALID_ARG;
+  if (transpose != 0 && transpose != 1) return MXATTN_ERR_INVALID_ARG;
+  if (batch == 0 || rows == 0 || cols == 0) return MXATTN_OK;
+  if (!x || !codes || !scales) return MXATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(codes, 16)) return MXATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int vec_ok = (aligned(x, 16) && cols % 8 == 0) ? 1 : 0;
+  if (transpose == 0) {
+    const uint64_t kb = (static_cast<uint64_t>(cols) + 31) / 32;
+    if (static_cast<uint64_t>(batch) * rows * kb >= (1ull << 31) || rows >= (1ll << 31) || cols >= (1ll << 31))
+      return MXATTN_ERR_UNSUPPORTED;
+    RowQuantParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.heads = static_cast<uint32_t>(batch);
+    p.rows = static_cast<uint32_t>(rows);
+    p.rows_pad = static_cast<uint32_t>(rows);
+    p.cols = static_cast<uint32_t>(cols);
+    p.kb = static_cast<uint32_t>(kb);
+    p.codes = codes;
+    p.scales = scales;
+    p.mode = scale_mode;
+    p.sf_layout = kSfRowMajor;
+    p.vec_ok = vec_ok;
+    return launch_quantize_rows(p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+  }
+  const uint64_t nblk = (static_cast<uint64_t>(rows) + 31) / 32;
+  if (batch > 65535 || static_cast<uint64_t>(batch) * cols * nblk >= (1ull << 31) || rows >= (1ll << 31) ||
+      cols >= (1ll << 31))
+    return MXATTN_ERR_UNSUPPORTED;
+  ColQuantParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.heads = static_cast<uint32_t>(batch);
+  p.rows = static_cast<uint32_t>(rows);
+  p.cols = static_cast<uint32_t>(cols);
+  p.nblk = static_cast<uint32_t>(nblk);
+  p.codes = codes;
+  p.scales = scales;
+  p.mode = scale_mode;
+  p.sf_layout = kSfRowMajor;
+  p.vec_ok = vec_ok;
+  return launch_quantize_cols(p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+size_t mxattn_forward_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  WsLayout L;
+  return ws_layout(B, Hq, Hkv, N, d, &L) ? L.total : 0;
+}
+
+mxattn_status mxattn_forward_prepare(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N,
+                                     int d, int scale_mode, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!q || !k || !v) return MXATTN_ERR_INVALID_ARG;
+  WsLayout L;
+  mxattn_status s = check_forward_args(q, k, v, nullptr, B, Hq, Hkv, N, d, scale_mode, MXATTN_OUT_F32, workspace,
+                                       workspace_bytes, &L);
+  if (s != MXATTN_OK) return s;
+  return prepare_impl(q, k, v, B, Hq, Hkv, N, d, scale_mode, workspace, workspace_bytes,
+                      static_cast<cudaStream_t>(stream), L);
+}
+
+mxattn_status mxattn_forward_attend(void* out, int B, int Hq, int Hkv, int N, int d, int causal, int scale_mode,
+                                    int pnq, int out_dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (!out) return MXATTN_ERR_INVALID_ARG;
+  WsLayout L;
+  mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, out, B, Hq, Hkv, N, d, scale_mode, out_dtype,
+                                       workspace, workspace_bytes, &L);
+  if (s != MXATTN_OK) return s;
+  return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace,
+                     static_cast<cudaStream_t>(stream), L, -1, 0, 0, nullptr, nullptr);
+}
+
+mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                             int N, int d, int causal, int scale_mode, int pnq, int out_dtype, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return mxattn_forward_debug(q, k, v, out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace,
+                              workspace_bytes, stream, -1, 0, 0, nullptr, nullptr);
+}
+
+mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                   int Hkv, int N, int d, int causal, int scale_mode, int pnq, int out_dtype,
+                                   void* workspace, size_t workspace_bytes, void* stream, int dbg_bh, int dbg_r0,
+                                   int dbg_r1, uint8_t* p_codes, uint8_t* p_scales) {
+  if (!q || !k || !v || !out) return MXATTN_ERR_INVALID_ARG;
+  WsLayout L;
+  mxattn_status s = check_forward_args(q, k, v, out, B, Hq, Hkv, N, d, scale_mode, out_dtype, workspace,
+                                       workspace_bytes, &L);
+  if (s != MXATTN_OK) return s;
+  if (p_codes || p_scales) {
+    if (!p_codes || !p_scales || dbg_bh < 0 || dbg_bh >= B * Hq || dbg_r0 < 0 || dbg_r1 <= dbg_r0 ||
+        dbg_r1 > L.npad || !aligned(p_codes, 16) || !aligned(p_scales, 4))
+      return MXATTN_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = prepare_impl(q, k, v, B, Hq, Hkv, N, d, scale_mode, workspace, workspace_bytes, st, L);
+  if (s != MXATTN_OK) return s;
+  return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace, st, L, dbg_bh, dbg_r0,
+                     dbg_r1, p_codes, p_scales);
+}
+
+mxattn_status mxattn_check_status(void* workspace, void* stream, unsigned int* detail) {
+  if (!workspace) return MXATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MXATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (detail) *detail = word;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    return MXATTN_ERR_TIMEOUT;
+  }
+  return MXATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Internal declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace mxattn {
+
+enum SfLayout : int { kSfRowMajor = 0, kSfAtom = 1 };
+
+// Blocks of 32 along the contiguous axis of `heads` matrices of [rows, cols] bf16. Rows in
+// [rows, rows_pad) are written as all-zero blocks (codes 0, scale byte 0).
+struct RowQuantParams {
+  const __nv_bfloat16* x;
+  uint32_t heads, rows, rows_pad, cols, kb;   // kb = ceil(cols / 32)
+  uint8_t* codes;                              // [heads][rows_pad][kb * 16]
+  uint8_t* scales;                             // row-major [heads][rows_pad][kb] or atom tiles
+  int mode;                                    // 0 = OCP, 1 = UOS
+  int sf_layout;
+  int vec_ok;                                  // cols % 8 == 0 and x 16-byte aligned
+};
+
+// Blocks of 32 along the row axis of `heads` matrices of [rows, cols] bf16, written
+// transposed: codes [heads][cols][nblk * 16], nblk >= ceil(rows / 32) (extra blocks are zero).
+struct ColQuantParams {
+  const __nv_bfloat16* x;
+  uint32_t heads, rows, cols, nblk;
+  uint8_t* codes;
+  uint8_t* scales;                             // row-major [heads][cols][nblk] or atom tiles
+  int mode;
+  int sf_layout;
+  int vec_ok;
+};
+
+cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream);
+cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
+
+struct AttnParams {
+  const uint8_t* qsf;      // atom-tiled scales of Q  [B*Hq][Npad/128][512]
+  const uint8_t* ksf;      // atom-tiled scales of K  [B*Hkv][Npad/128][512]
+  const uint8_t* vsf;      // atom-tiled scales of V^T [B*Hkv][Npad/128][512]
+  void* out;               // [B, Hq, N, d], fp32 or bf16
+  int out_bf16;
+  int B, Hq, Hkv, N, Npad, causal, mode, pnq;
+  float scale_log2;        // log2(e) / sqrt(d)
+  unsigned int* status;    // device status word (0 = ok)
+  uint8_t* dbg_codes;      // optional P~ dump: [r1 - r0][Npad / 2]
+  uint8_t* dbg_scales;     //                  [r1 - r0][Npad / 32]
+  int dbg_bh, dbg_r0, dbg_r1;
+};
+
+cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                             const AttnParams& p, int d, cudaStream_t stream);
+
+// Status codes written by kernels into the workspace status word.
+enum : unsigned int {
+  kStatusTimeoutQ = 0x100,
+  kStatusTimeoutKV = 0x200,
+  kStatusTimeoutS = 0x300,
+  kStatusTimeoutP = 0x400,
+  kStatusTimeoutPV = 0x500,
+  kStatusTimeoutEmpty = 0x600,
+};
+
+}  // namespace mxattn

@@ -1,0 +1,199 @@
+// MXFP4 block quantizer kernels (bf16 -> packed E2M1 codes + E8M0 scales).
+//
+// Method: "Quantization Error" page, section "Where the error comes from" (one rounding step
+// onto eight E2M1 magnitudes, an exact power-of-two scale per block, no dependence on block
+// order) and the MXAttention abstract (Universal Optimal Scaling, Qmax = 7.25, next to the OCP
+// rule). Each 32-element block: amax -> shared exponent (OCP or UOS) -> x * 2^-e rounded to
+// nearest-even on the E2M1 grid, saturating at 6, by the hardware conversion
+// cvt.rn.satfinite.e2m1x2.f32.
+//
+// Two kernels:
+//  * quantize_rows_kernel: blocks along the contiguous axis (Q, K, the standalone tensor). One
+//    thread owns one whole block: four 16-byte loads, a thread-local amax, one 16-byte store of
+//    codes. A warp therefore reads 2 KiB and writes 512 B of codes per step, fully coalesced.
+//  * quantize_cols_kernel: blocks along the row axis of a [R, C] matrix, written transposed as
+//    [C, R/2] codes (V along keys). A CTA stages 256 rows x 64 columns in shared memory; each
+//    thread then quantizes two consecutive 32-row blocks of one column and writes 32 contiguous
+//    bytes of codes.
+//
+// Scale placement: row-major [.., rows, blocks] (the library's canonical layout), or the tile
+// layout the block-scaled tensor-core MMA consumes: per 128-row tile and 4 blocks along K, a
+// 512-byte atom where the byte of (row r, block k) sits at (r % 32) * 16 + (r / 32) * 4 + k.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "mxattn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace mxattn {
+
+__device__ __forceinline__ uint32_t atom_offset(uint32_t r128, uint32_t k4) {
+  return (r128 & 31u) * 16u + (r128 >> 5) * 4u + k4;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float* v) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Quantize 32 fp32 values (one block) into 16 code bytes and return the scale byte.
+__device__ __forceinline__ uint32_t quantize_block32(float* v, int mode, uint4& codes) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t byte = e8m0_scale_byte(amax, mode);
+  const float inv = inv_pow2_from_byte(byte);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= inv;   // exact: power of two
+  codes.x = cvt_e2m1x8(v);
+  codes.y = cvt_e2m1x8(v + 8);
+  codes.z = cvt_e2m1x8(v + 16);
+  codes.w = cvt_e2m1x8(v + 24);
+  return byte;
+}
+
+__global__ void __launch_bounds__(256) quantize_rows_kernel(RowQuantParams p) {
+  const uint32_t total = p.heads * p.rows_pad * p.kb;   // blocks
+  const uint32_t row_bytes = p.kb * 16u;
+  for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x) {
+    const uint32_t row = g / p.kb;               // head * rows_pad + n
+    const uint32_t kbi = g - row * p.kb;
+    const uint32_t head = row / p.rows_pad;
+    const uint32_t n = row - head * p.rows_pad;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    if (n < p.rows) {
+      const uint64_t src_row = static_cast<uint64_t>(head) * p.rows + n;
+      const __nv_bfloat16* src = p.x + src_row * p.cols + static_cast<uint64_t>(kbi) * 32u;
+      const uint32_t c0 = kbi * 32u;
+      if (p.vec_ok && c0 + 32u <= p.cols) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) bf16x8_to_f32(ld_stream_u4(src + 8 * c), v + 8 * c);
+      } else {
+        for (uint32_t i = 0; i < 32u && c0 + i < p.cols; ++i) v[i] = __bfloat162float(src[i]);
+      }
+    }
+    uint4 codes;
+    const uint32_t byte = quantize_block32(v, p.mode, codes);
+    *reinterpret_cast<uint4*>(p.codes + static_cast<uint64_t>(row) * row_bytes + kbi * 16u) = codes;
+    uint64_t so;
+    if (p.sf_layout == kSfRowMajor) {
+      so = static_cast<uint64_t>(row) * p.kb + kbi;
+    } else {
+      const uint32_t tiles = p.rows_pad >> 7;
+      const uint32_t katoms = (p.kb + 3u) >> 2;
+      const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (n >> 7)) * katoms + (kbi >> 2);
+      so = atom * 512u + atom_offset(n & 127u, kbi & 3u);
+    }
+    p.scales[so] = static_cast<uint8_t>(byte);
+  }
+}
+
+// Stage: 256 rows x 64 columns of bf16, row pitch 72 elements (144 B) so that the column reads
+// of the compute phase (32 lanes on consecutive columns) hit distinct banks.
+constexpr int kColTileRows = 256;
+constexpr int kColTileCols = 64;
+constexpr int kColPitch = 72;
+
+__global__ void __launch_bounds__(256) quantize_cols_kernel(ColQuantParams p) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kColTileRows * kColPitch];
+  const uint32_t head = blockIdx.z;
+  const uint32_t r0 = blockIdx.x * kColTileRows;      // first row (key) of this tile
+  const uint32_t c0 = blockIdx.y * kColTileCols;      // first column (channel)
+  const __nv_bfloat16* src = p.x + static_cast<uint64_t>(head) * p.rows * p.cols;
+  const int tid = threadIdx.x;
+
+  // Load: each pass covers 32 rows x 64 columns, one 16-byte vector per thread.
+#pragma unroll 4
+  for (int pass = 0; pass < kColTileRows / 32; ++pass) {
+    const uint32_t rr = pass * 32 + (tid >> 3);
+    const uint32_t cc = (tid & 7) * 8;
+    const uint32_t r = r0 + rr, c = c0 + cc;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (r < p.rows) {
+      const __nv_bfloat16* s = src + static_cast<uint64_t>(r) * p.cols + c;
+      if (p.vec_ok && c + 8 <= p.cols) {
+        raw = ld_stream_u4(s);
+      } else {
+        uint16_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (uint32_t i = 0; i < 8 && c + i < p.cols; ++i) h[i] = __bfloat16_as_ushort(s[i]);
+        raw.x = h[0] | (uint32_t(h[1]) << 16);
+        raw.y = h[2] | (uint32_t(h[3]) << 16);
+        raw.z = h[4] | (uint32_t(h[5]) << 16);
+        raw.w = h[6] | (uint32_t(h[7]) << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(&tile[rr * kColPitch + cc]) = raw;
+  }
+  __syncthreads();
+
+  // Compute: thread (column cl, pair kp) quantizes row blocks 2kp and 2kp+1 of its column.
+  const uint32_t cl = tid & 63;
+  const uint32_t kp = tid >> 6;
+  const uint32_t col = c0 + cl;
+  const uint32_t blk0 = (r0 >> 5) + 2 * kp;          // absolute block index along rows
+  if (col >= p.cols || blk0 >= p.nblk) return;
+  uint4 codes[2];
+  uint32_t bytes[2];
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    float v[32];
+    const uint32_t rb = (2 * kp + b) * 32;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[(rb + i) * kColPitch + cl]);
+    bytes[b] = quantize_block32(v, p.mode, codes[b]);
+  }
+  const bool second = blk0 + 1 < p.nblk;
+  uint8_t* dst = p.codes + (static_cast<uint64_t>(head) * p.cols + col) * (p.nblk * 16u) + blk0 * 16u;
+  reinterpret_cast<uint4*>(dst)[0] = codes[0];
+  if (second) reinterpret_cast<uint4*>(dst)[1] = codes[1];
+  if (p.sf_layout == kSfRowMajor) {
+    uint8_t* s = p.scales + (static_cast<uint64_t>(head) * p.cols + col) * p.nblk + blk0;
+    s[0] = static_cast<uint8_t>(bytes[0]);
+    if (second) s[1] = static_cast<uint8_t>(bytes[1]);
+  } else {
+    // atom per (head, 128-row tile, 128-column group); MN index = column, K index = block
+    const uint32_t tiles = p.nblk >> 2;               // nblk is a multiple of 4 here
+    const uint32_t cgroups = (p.cols + 127u) >> 7;
+    const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (blk0 >> 2)) * cgroups + (col >> 7);
+    uint8_t* s = p.scales + atom * 512u + atom_offset(col & 127u, blk0 & 3u);
+    s[0] = static_cast<uint8_t>(bytes[0]);
+    if (second) s[1] = static_cast<uint8_t>(bytes[1]);
+  }
+}
+
+cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream) {
+  const uint64_t total = static_cast<uint64_t>(p.heads) * p.rows_pad * p.kb;
+  if (total == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t want = (total + 255) / 256;
+  const uint64_t cap = static_cast<uint64_t>(sms) * 8;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  quantize_rows_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream) {
+  if (p.heads == 0 || p.cols == 0 || p.nblk == 0) return cudaSuccess;
+  dim3 grid((p.nblk * 32u + kColTileRows - 1) / kColTileRows, (p.cols + kColTileCols - 1) / kColTileCols,
+            p.heads);
+  quantize_cols_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mxattn

@@ -1,0 +1,110 @@
+"""CPU-side checks of the C ABI: the library builds and loads without a GPU, exports every
+function include/mxattn.h declares, and rejects bad arguments on the host before any CUDA call."""
+import os
+import re
+
+import pytest
+
+from mxfp4_microscaled_bit_quantize_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxattn.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 0x100000  # aligned non-null address; never dereferenced by the host-side checks
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxattn_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.mxattn_version() >= 100
+    assert lib.mxattn_status_string(0) == b"ok"
+    assert lib.mxattn_status_string(5) == b"device pipeline timeout"
+    assert lib.mxattn_status_string(99) == b"unknown status"
+
+
+def test_quantize_argument_checks(lib):
+    q = lib.mxattn_quantize
+    assert q(None, 0, 10, 10, 0, 1, None, None, None) == OK          # empty: no-op
+    assert q(None, 1, 10, 10, 0, 1, None, None, None) == INVALID
+    assert q(FAKE, 1, 10, 10, 0, 7, FAKE, FAKE, None) == INVALID        # bad mode
+    assert q(FAKE, 1, 10, 10, 2, 1, FAKE, FAKE, None) == INVALID        # bad transpose flag
+    assert q(FAKE + 1, 1, 10, 10, 0, 1, FAKE, FAKE, None) == INVALID    # misaligned x
+    assert q(FAKE, 1, 10, 10, 0, 1, FAKE + 8, FAKE, None) == INVALID    # misaligned codes
+    assert q(FAKE, -1, 10, 10, 0, 1, FAKE, FAKE, None) == INVALID
+    assert q(FAKE, 70000, 32, 32, 1, 1, FAKE, FAKE, None) == UNSUPPORTED
+    assert q(FAKE, 1 << 20, 1 << 20, 1024, 0, 1, FAKE, FAKE, None) == UNSUPPORTED
+
+
+def _ws_mirror(B, Hq, Hkv, N, d):
+    up = lambda x, a: -(-x // a) * a  # noqa: E731
+    npad = up(N, 128)
+    t = npad // 128
+    off = 1024
+    for nbytes in (B * Hq * npad * d // 2, B * Hq * t * 512, B * Hkv * npad * d // 2, B * Hkv * t * 512,
+                   B * Hkv * d * npad // 2, B * Hkv * t * 512):
+        off = up(off + nbytes, 1024)
+    return off
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 256, 64), (1, 40, 40, 32760, 128), (4, 32, 8, 8192, 128),
+                                   (1, 24, 24, 76800, 128), (2, 3, 1, 1, 64)])
+def test_workspace_size(lib, shape):
+    assert lib.mxattn_forward_workspace_size(*shape) == _ws_mirror(*shape)
+
+
+def test_workspace_size_rejects_bad_shapes(lib):
+    ws = lib.mxattn_forward_workspace_size
+    assert ws(1, 2, 2, 256, 96) == 0
+    assert ws(1, 3, 2, 256, 64) == 0
+    assert ws(1, 2, 2, 0, 64) == 0
+
+
+def test_forward_argument_checks(lib):
+    f = lib.mxattn_forward
+    good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
+    args = lambda **kw: dict(dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, Hq=2, Hkv=2, N=256, d=64,  # noqa: E731
+                                  causal=0, mode=1, pnq=1, od=0, ws=FAKE, wsb=good, st=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["causal"],
+                 a["mode"], a["pnq"], a["od"], a["ws"], a["wsb"], a["st"])
+
+    assert call(d=96) == UNSUPPORTED
+    assert call(Hq=3) == INVALID
+    assert call(N=0) == INVALID
+    assert call(mode=2) == INVALID
+    assert call(od=5) == INVALID
+    assert call(q=None) == INVALID
+    assert call(q=FAKE + 2) == INVALID
+    assert call(ws=FAKE + 16) == INVALID
+    assert call(wsb=good - 1) == WORKSPACE
+
+
+def test_debug_argument_checks(lib):
+    good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
+    r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
+                                 5, 0, 16, FAKE, FAKE)   # head index out of range
+    assert r == INVALID
+    r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
+                                 0, 10, 5, FAKE, FAKE)   # empty row range
+    assert r == INVALID
