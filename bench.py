@@ -113,8 +113,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def reduce_max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tflops(flops_per_rank: float, world: int, step_ms: float) -> float:
+    """Whole-job throughput: every rank processed its own problem in at most step_ms."""
+    return world * flops_per_rank / (step_ms * 1e-3) / 1e12
+
+
 def oracle_sample(cfg, rows: int, head: int = 0):
-    """CPU oracle on a bounded sample: quantize one head's Q/K/V, then `rows` query rows of it."""
+    """CPU oracle on a bounded sample: quantize one head's Q/K/V, then attend `rows` query rows of it
+    over all keys. Returns (algorithmic FLOP of those rows, seconds)."""
     from mxfp4_microscaled_bit_quantize_b200 import synthetic
     from oracle import attention as oa
     from oracle import mxfp4 as mx
@@ -124,9 +140,9 @@ def oracle_sample(cfg, rows: int, head: int = 0):
     k = synthetic.head_bf16(cfg, "k", 0, g).double().numpy()
     v = synthetic.head_bf16(cfg, "v", 0, g).double().numpy()
     t0 = time.perf_counter()
-    (qd, kd, vd), _ = oa.dequantized_qkv(q[:rows], k, v, mx.SCALE_UOS)
+    (qd, kd, vd), _ = oa.dequantized_qkv(q, k, v, mx.SCALE_UOS)
     idx = np.arange(rows)
-    oa.attention_rows(qd, idx, kd, vd, causal=cfg.causal, mode=mx.SCALE_UOS, pnq=True)
+    oa.attention_rows(qd[:rows], idx, kd, vd, causal=cfg.causal, mode=mx.SCALE_UOS, pnq=True)
     dt = time.perf_counter() - t0
     flops = 4.0 * rows * cfg.N * cfg.d / (2.0 if cfg.causal else 1.0)
     return flops, dt
@@ -178,7 +194,12 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = synthetic.ATTN_CONFIGS[WORKLOAD]
+    if args.heads:
+        cfg = cfg.scaled(Hq=args.heads, Hkv=args.heads)
     B, Hq, Hkv, N, d = cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.d
+    if args.mode == "quantizer":
+        run_quantizer_only(args, dev)
+        return
     q, k, v = synthetic.attn_inputs(cfg)
     q_h, k_h, v_h = (t.pin_memory() for t in (q, k, v))
     dq, dk, dv = (t.to(dev) for t in (q_h, k_h, v_h))
@@ -219,6 +240,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     total_ms = start.elapsed_time(stop)
     quant_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    if args.mode == "attention":
+        print(json.dumps({"mode": "attention", "config": cfg.describe(), "attn_ms": attn_ms,
+                          "quant_ms": quant_ms, "tflops": cfg.flops / (attn_ms * 1e-3) / 1e12}), flush=True)
+        return
 
     # end to end through the public call with host buffers: H2D inputs, forward, D2H output
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
@@ -255,10 +280,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
-    vals = torch.tensor([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms = (float(x) for x in vals.tolist())
+    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms = reduce_max_over_ranks(
+        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms], world, dev)
     if rank != 0:
         return
 
@@ -273,7 +296,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     qa_bytes = qa_elems * 2 + qa_elems // 2 + qa_elems // 32
     line = {
         "metric": METRIC,
-        "value": world * flops / (step_ms * 1e-3) / 1e12,
+        "value": job_tflops(flops, world, step_ms),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -297,7 +320,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                       "standalone_ms": quant_alone_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
                       "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks.summary(),
@@ -311,15 +334,39 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_quantizer_only(args, dev):
+    """The standalone quantizer workload alone (used for its Nsight Compute capture)."""
+    import torch
+
+    from mxfp4_microscaled_bit_quantize_b200 import api, synthetic
+    xq = [synthetic.quant_input().to(dev) for _ in range(2)]
+    for i in range(args.warmup):
+        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(args.steps):
+        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
+    e.record()
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / args.steps
+    n = xq[0].numel()
+    gbs = (n * 2 + n // 2 + n // 32) / (ms * 1e-3) / 1e9
+    print(json.dumps({"mode": "quantizer", "ms": ms, "gbs": gbs}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=128)
-    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["full", "attention", "quantizer"], default="full",
+                    help="attention / quantizer: time only that part (small cases for profiling)")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
