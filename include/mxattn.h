@@ -122,6 +122,29 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
                                    int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales);
 
 /*
+ * mxattn_forward_noalloc -- mxattn_forward for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it exists for deployment. Some callers
+ * cannot call cudaMalloc: code whose device memory is owned by a host process or framework
+ * (an inference server or plugin host with a fixed arena, an allocator that must account for
+ * every byte), or a latency-critical loop where an allocation call, which may synchronise the
+ * device or fail when a memory pool holds the free memory, is not allowed. They still pass
+ * q, k, v and out exactly as for mxattn_forward; the workspace instead comes from a static
+ * device array of MXATTN_NOALLOC_MAX_WORKSPACE bytes that every GPU loading the library holds
+ * until the process exits.
+ *   - Shapes with mxattn_forward_workspace_size(...) > MXATTN_NOALLOC_MAX_WORKSPACE are rejected
+ *     with MXATTN_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device (that device current) looks up the array's device address;
+ *     make it before any stream capture. No call allocates.
+ *   - All calls on a device share the array: calls whose kernels overlap on the GPU race, so
+ *     serialise them (one stream, or explicit ordering). The status word is cleared at the
+ *     start of each call; device-side timeouts are not reported by this entry point.
+ */
+#define MXATTN_NOALLOC_MAX_WORKSPACE ((size_t)16 << 20)
+mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                     int Hkv, int N, int d, int causal, int scale_mode, int pnq, int out_dtype,
+                                     void* stream);
+
+/*
  * mxattn_check_status -- synchronises `stream`, reads and clears the workspace status word.
  * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last check (the
  * raw code goes to *detail when detail != NULL), MXATTN_ERR_CUDA on a CUDA error, else MXATTN_OK.

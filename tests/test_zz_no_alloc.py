@@ -1,0 +1,78 @@
+"""mxattn_forward_noalloc: the attention forward for callers that cannot allocate device memory
+(a host or framework that owns all device memory, or a loop where an allocation call is not
+allowed). It takes the workspace from a static device array inside the library instead of a
+caller buffer. This file is collected last on purpose.
+
+Checks, through the C ABI: two calls in a row each match mxattn_forward (the entry point with a
+caller-provided workspace) within the parity tolerances, and a shape whose workspace exceeds
+the static array is rejected before anything runs.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from mxfp4_microscaled_bit_quantize_b200 import _lib, api, build, synthetic
+from oracle import mxfp4 as mx
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+MAX_WORKSPACE = 16 << 20       # MXATTN_NOALLOC_MAX_WORKSPACE in include/mxattn.h
+WORKSPACE_ERR = 3              # MXATTN_ERR_WORKSPACE
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    return _lib.load()
+
+
+def _noalloc(lib, q, k, v, out, causal, mode, pnq):
+    B, Hq, N, d = q.shape
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    return lib.mxattn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
+                                      k.shape[1], N, d, int(causal), mode, int(pnq), 0, stream)
+
+
+@pytest.mark.parametrize("mode,pnq,causal", [(mx.SCALE_UOS, True, False), (mx.SCALE_OCP, False, True)])
+def test_noalloc_matches_forward_twice(lib, mode, pnq, causal):
+    dev = torch.device("cuda:0")
+    cfg = synthetic.ATTN_CONFIGS["tiny"]
+    q, k, v = (t.to(dev) for t in synthetic.attn_inputs(cfg))
+    assert lib.mxattn_forward_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.d) <= MAX_WORKSPACE
+    ref = api.mxattn_forward(q, k, v, causal=causal, scale_mode=mode, pnq=pnq).cpu().numpy()
+    for _ in range(2):
+        out = torch.full(q.shape, float("nan"), dtype=torch.float32, device=dev)
+        assert _noalloc(lib, q, k, v, out, causal, mode, pnq) == 0
+        torch.cuda.synchronize()
+        got = out.cpu().numpy()
+        assert np.isfinite(got).all()
+        mabs, rfro = parity.out_errors(got, ref)
+        assert mabs <= parity.OUT_MAX_ABS and rfro <= parity.OUT_REL_FRO, (mabs, rfro)
+
+
+def test_noalloc_other_shape_after_first(lib):
+    # a second shape through the same static array (d = 128, GQA, ragged N)
+    dev = torch.device("cuda:0")
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(1, 4, 300, 128, generator=g).bfloat16().to(dev)
+    k = torch.randn(1, 2, 300, 128, generator=g).bfloat16().to(dev)
+    v = torch.randn(1, 2, 300, 128, generator=g).bfloat16().to(dev)
+    ref = api.mxattn_forward(q, k, v, causal=True).cpu().numpy()
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    assert _noalloc(lib, q, k, v, out, True, mx.SCALE_UOS, True) == 0
+    torch.cuda.synchronize()
+    mabs, rfro = parity.out_errors(out.cpu().numpy(), ref)
+    assert mabs <= parity.OUT_MAX_ABS and rfro <= parity.OUT_REL_FRO, (mabs, rfro)
+
+
+def test_noalloc_rejects_oversize(lib):
+    # video-DiT shape needs ~267 MB of workspace, far beyond the static array: rejected on the host
+    assert lib.mxattn_forward_workspace_size(1, 40, 40, 32760, 128) > MAX_WORKSPACE
+    fake = ctypes.c_void_p(0x100000)
+    r = lib.mxattn_forward_noalloc(fake, fake, fake, fake, 1, 40, 40, 32760, 128, 0, 1, 1, 0, None)
+    assert r == WORKSPACE_ERR
