@@ -14,9 +14,10 @@
  *       MXATTN_SCALE_UOS: smallest e with amax / 2^e <= 7.25 (Universal Optimal Scaling)
  *     An all-zero block gets scale byte 0 and all-zero codes.
  *   - Attention: Q, K quantized along the head dimension, V along keys; S = Q K^T as a
- *     block-scaled FP4 contraction; FlashAttention online softmax over 128-key tiles in
- *     increasing key order (running max, history rescale, fp32 accumulation, final
- *     normalisation; "EFQ-Softmax" abstract). With pnq = 1 (Pre-Normalization Quantization)
+ *     block-scaled FP4 contraction; FlashAttention online softmax over key tiles of
+ *     MXATTN_KV_TILE keys in increasing key order (running max, history rescale, fp32
+ *     accumulation, final normalisation; "EFQ-Softmax" abstract).
+ *     With pnq = 1 (Pre-Normalization Quantization)
  *     the unnormalised exponentials P~ = exp(S/sqrt(d) - m) are quantized to MXFP4 along keys
  *     before the row sum, and that same dequantized operand feeds both P~V and the row sum.
  *     With pnq = 0 the row sum uses the unquantized fp32 P~ (exp-then-quantize baseline).
@@ -46,6 +47,10 @@ extern "C" {
 #endif
 
 typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1 } mxattn_scale_mode;
+
+/* Keys per tile of the online softmax. P~ is quantized with the running max in force at each
+ * tile, so the tile width is part of the result (a CPU reference must use the same width). */
+#define MXATTN_KV_TILE 64
 
 typedef enum { MXATTN_OUT_F32 = 0, MXATTN_OUT_BF16 = 1 } mxattn_out_dtype;
 

@@ -12,7 +12,8 @@ from . import _lib
 
 SCALE_OCP, SCALE_UOS = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
-KV_TILE = 128
+KV_TILE = 64          # keys per online-softmax tile (MXATTN_KV_TILE)
+NPAD_ALIGN = 128      # the workspace pads N to a multiple of this
 
 
 def _stream(dev: torch.device) -> int:
@@ -29,7 +30,7 @@ def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16) -> None:
 
 
 def npad(N: int) -> int:
-    return -(-N // KV_TILE) * KV_TILE
+    return -(-N // NPAD_ALIGN) * NPAD_ALIGN
 
 
 def mxattn_quantize(x: torch.Tensor, transpose: bool = False, scale_mode: int = SCALE_UOS):

@@ -13,20 +13,23 @@
 //   pnq = 0 keeps the conventional path: l sums the unquantized fp32 P~ on the CUDA cores.
 //   out = O / l.
 //
-// One CTA owns one 128-query tile of one (batch, query head); keys are visited in tiles of 128
-// in increasing order (P~ codes depend on the running max in force, so the order is part of
-// the definition). Warp roles (256 threads):
-//   warp 0     TMA producer: Q tile once, then K / V^T tiles and their scale atoms into a
+// One CTA owns one 128-query tile of one (batch, query head) and visits keys in tiles of
+// kKvTile = 64 in increasing order (P~ codes depend on the running max in force, so tile width
+// and order are part of the definition; the oracle takes the same width). Two CTAs share an SM:
+// each allocates half of TMEM and their softmax phases drift apart, so one CTA's exponentials
+// overlap the other's serial work (max, scale selection, stores, rescale).
+// Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile once, then K / V^T tiles and their scale atoms into an
 //              NSTAGE-deep shared-memory ring (mbarrier complete_tx).
-//   warp 1     TMEM owner and MMA issuer (one elected thread): copies scale atoms to TMEM with
-//              tcgen05.cp, issues S = QK^T into one of two S buffers and O += P~ V^T.
-//   warps 4-7  softmax warpgroup, one thread per query row (TMEM lane = row): reads S with
-//              tcgen05.ld, updates the running max, computes P~, quantizes it in registers,
-//              writes codes (64B-swizzled, the MMA operand layout) and scale atoms to shared
-//              memory, keeps the row sum, rescales O in TMEM when the max moves, and finally
-//              normalises and stores the output.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+d) row sum L [384,400), scale atoms at
-// 400..419 (Q, K, V, P~, ones).
+//   warp 1     TMEM owner and MMA issuer (one thread): copies scale atoms to TMEM with
+//              tcgen05.cp, issues S = QK^T, O += P~ V^T and (PNQ) L += P~ 1.
+//   warps 2-5  softmax warpgroup, one thread per query row (TMEM lane = row): reads S with
+//              tcgen05.ld (S is single-buffered: the MMA for the next tile starts as soon as the
+//              row is in registers), updates the running max, computes P~ / 2^e per 32-key block,
+//              quantizes it in registers, writes codes (32B-swizzled, the MMA operand layout)
+//              and scale bytes to shared memory, rescales O and L in TMEM when the max moves,
+//              and finally normalises and stores the output.
+// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..231.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -37,22 +40,24 @@
 namespace mxattn {
 
 constexpr int kBM = 128;          // query rows per CTA
-constexpr int kBN = 128;          // keys per KV tile
-constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColL = 384;
-constexpr uint32_t kColSfQ = 400, kColSfK = 404, kColSfV = 408, kColSfP = 412, kColSf1 = 416;
+constexpr int kBN = kKvTile;      // keys per KV tile (64)
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColO = 64, kColL = 192;
+constexpr uint32_t kColSfQ = 208, kColSfK = 212, kColSfV = 216, kColSfP = 220, kColSf1 = 224;
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
-constexpr size_t kMinSmem = 120 * 1024;   // keeps one CTA per SM (its TMEM allocation is 512)
+constexpr int kPRowBytes = kBN / 2;                  // 32 bytes of codes per P~ row
+constexpr size_t kMinSmem = 80 * 1024;               // at most two CTAs per SM (TMEM halves)
+
+static_assert(kBN == 64, "the 32B-swizzled P~ / V^T layouts below assume 64-key tiles");
 
 template <int D>
 struct Cfg {
-  static constexpr int kStages = 6;
+  static constexpr int kStages = 8;
   static constexpr int kQRowBytes = D / 2;                 // packed E2M1 per Q/K row
   static constexpr int kQTileBytes = kBM * kQRowBytes;
   static constexpr int kKTileBytes = kBN * kQRowBytes;
-  static constexpr int kVTileBytes = D * (kBN / 2);        // V^T: D rows of 128 keys
-  static constexpr int kPTileBytes = kBM * (kBN / 2);
+  static constexpr int kVTileBytes = D * kPRowBytes;       // V^T: D rows of 64 keys
   static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
   static constexpr uint32_t kQKSbo = 8 * kQRowBytes;       // 8-row swizzle atom
 };
@@ -62,8 +67,8 @@ struct __align__(1024) Smem {
   uint8_t q[Cfg<D>::kQTileBytes];
   uint8_t k[Cfg<D>::kStages][Cfg<D>::kKTileBytes];
   uint8_t v[Cfg<D>::kStages][Cfg<D>::kVTileBytes];
-  uint8_t p[Cfg<D>::kPTileBytes];
-  uint8_t ones[kOnesRows * (kBN / 2)];
+  uint8_t p[kBM * kPRowBytes];
+  uint8_t ones[kOnesRows * kPRowBytes];
   uint8_t qsf[512];
   uint8_t ksf[Cfg<D>::kStages][512];
   uint8_t vsf[Cfg<D>::kStages][512];
@@ -72,8 +77,8 @@ struct __align__(1024) Smem {
   uint64_t bar_q;
   uint64_t bar_kv_full[Cfg<D>::kStages];
   uint64_t bar_kv_empty[Cfg<D>::kStages];
-  uint64_t bar_s_full[2];
-  uint64_t bar_s_empty[2];
+  uint64_t bar_s_full;
+  uint64_t bar_s_empty;
   uint64_t bar_p_full;
   uint64_t bar_pv_done;
   uint64_t bar_drain;
@@ -106,8 +111,26 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+// max over 32 consecutive values with three-input max instructions
+__device__ __forceinline__ float block_max32(const float* v) {
+  float a0 = fmax3(v[0], v[1], v[2]);
+  float a1 = fmax3(v[3], v[4], v[5]);
+  float a2 = fmax3(v[6], v[7], v[8]);
+  float a3 = fmax3(v[9], v[10], v[11]);
+#pragma unroll
+  for (int i = 12; i < 28; i += 8) {          // elements 12..27
+    a0 = fmax3(a0, v[i], v[i + 1]);
+    a1 = fmax3(a1, v[i + 2], v[i + 3]);
+    a2 = fmax3(a2, v[i + 4], v[i + 5]);
+    a3 = fmax3(a3, v[i + 6], v[i + 7]);
+  }
+  a0 = fmax3(a0, v[28], v[29]);                // elements 28..31
+  a1 = fmax3(a1, v[30], v[31]);
+  return fmaxf(fmax3(a0, a1, a2), a3);
+}
+
+template <int D, bool PNQ>
+__global__ void __launch_bounds__(kThreads, 2)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = Cfg<D>;
@@ -131,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh_kv = b * p.Hkv + h / group;
   if (p.causal) qt = n_qt - 1 - qt;
   const int n_kv_all = p.Npad / kBN;
-  const int n_kv = p.causal ? min(qt + 1, n_kv_all) : n_kv_all;
+  const int n_kv = p.causal ? min(2 * qt + 2, n_kv_all) : n_kv_all;
 
   if (threadIdx.x == 0) {
     mbar_init(&s.bar_q, 1);
@@ -139,11 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_kv_full[i], 1);
       mbar_init(&s.bar_kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.bar_s_full[i], 1);
-      mbar_init(&s.bar_s_empty[i], 128);
-    }
-    mbar_init(&s.bar_p_full, 128);
+    mbar_init(&s.bar_s_full, 1);
+    mbar_init(&s.bar_s_empty, kBM);
+    mbar_init(&s.bar_p_full, kBM);
     mbar_init(&s.bar_pv_done, 1);
     mbar_init(&s.bar_drain, 1);
     s.abort_flag = 0;
@@ -178,8 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + 1024);
         tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.Npad + j * kBN);
-        tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * (kBN / 2), bh_kv * D);
-        const size_t atom = (static_cast<size_t>(bh_kv) * n_kv_all + j) * 512;
+        tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
+        // scale atoms cover 128 keys: tiles 2t and 2t+1 share atom t
+        const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;
         bulk_load(s.ksf[st], p.ksf + atom, 512, &s.bar_kv_full[st]);
         bulk_load(s.vsf[st], p.vsf + atom, 512, &s.bar_kv_full[st]);
         issued = j + 1;
@@ -196,10 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
       auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
-      if (p.pnq) {
+      if (PNQ) {
         // ones operand (row 0 = code 1.0 for every key, rows 1..15 = 0) with unit scales
         uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
-        for (int i = 0; i < kOnesRows * (kBN / 2) / 4; ++i) ow[i] = (i < (kBN / 2) / 4) ? 0x22222222u : 0u;
+        for (int i = 0; i < kOnesRows * kPRowBytes / 4; ++i) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
         uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
         for (int i = 0; i < 512 / 4; ++i) sw[i] = 0x7F7F7F7Fu;
         fence_proxy_async_smem();
@@ -208,27 +230,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         tc_cp_sf(tmem + kColSfQ, sf_desc(s.qsf));
-        if (p.pnq) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
+        if (PNQ) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
       }
       auto issue_s = [&](int j) -> bool {
         const int st = j % NS;
-        const int sb = j & 1;
         if (!mbar_wait(&s.bar_kv_full[st], (j / NS) & 1, abort_flag, p.status, kStatusTimeoutKV | st))
           return false;
-        if (j >= 2 && !mbar_wait(&s.bar_s_empty[sb], ((j >> 1) - 1) & 1, abort_flag, p.status,
-                                 kStatusTimeoutS | sb))
+        // S is single-buffered: the previous tile must be in the softmax registers
+        if (j >= 1 && !mbar_wait(&s.bar_s_empty, (j - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
           return false;
         tc_fence_after();
         tc_cp_sf(tmem + kColSfK, sf_desc(s.ksf[st]));
         const uint32_t qa = smem_u32(s.q), ka = smem_u32(s.k[st]);
+        // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
+        const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
           const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
           const uint64_t bd = smem_desc(ka + kk * 32, 0, C::kQKSbo, C::kQKLayout);
-          tc_mma_mxf4(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk),
-                      tmem + kColSfQ, tmem + kColSfK, kk > 0);
+          tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ, sfk, kk > 0);
         }
-        tc_commit(&s.bar_s_full[sb]);
+        tc_commit(&s.bar_s_full);
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
@@ -238,22 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_cp_sf(tmem + kColSfP, sf_desc(s.psf));
         tc_cp_sf(tmem + kColSfV, sf_desc(s.vsf[st]));
         const uint32_t pa = smem_u32(s.p), va = smem_u32(s.v[st]);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 64; ++kk) {
-          const uint64_t ad = smem_desc(pa + kk * 32, 0, 512, kLayoutSw64);
-          const uint64_t bd = smem_desc(va + kk * 32, 0, 512, kLayoutSw64);
-          tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 2 * kk, 2 * kk), tmem + kColSfP, tmem + kColSfV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        if (p.pnq) {
-          const uint32_t oa = smem_u32(s.ones);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 64; ++kk) {
-            const uint64_t ad = smem_desc(pa + kk * 32, 0, 512, kLayoutSw64);
-            const uint64_t bd = smem_desc(oa + kk * 32, 0, 512, kLayoutSw64);
-            tc_mma_mxf4(tmem + kColL, ad, bd, idesc_mxf4(kOnesRows, 2 * kk, 2 * kk), tmem + kColSfP,
-                        tmem + kColSf1, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+        const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
+        const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
+        // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
+        tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), tmem + kColSfP, tmem + kColSfV,
+                    j > 0 ? 1u : 0u);
+        if (PNQ) {
+          const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
+          tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), tmem + kColSfP, tmem + kColSf1,
+                      j > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_pv_done);
         tc_commit(&s.bar_kv_empty[st]);
@@ -268,23 +283,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&s.bar_drain);
       drain_wait(&s.bar_drain, 0);
     }
-  } else if (warp >= 4) {
+  } else {
     // ============================ softmax warpgroup ============================
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;                // row inside the tile == TMEM lane
     const int qrow = qt * kBM + r;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const float c = p.scale_log2;
     float m = -INFINITY;      // running max of the raw scores S
-    float l = 0.f;            // running row sum
+    float l = 0.f;            // running row sum (pnq = 0)
     bool ok = true;
     const bool dbg = p.dbg_codes != nullptr && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
-    uint8_t* p_row = s.p + r * (kBN / 2);
-    const uint32_t swz = (static_cast<uint32_t>(r) >> 1) & 3u;
+    uint8_t* p_row = s.p + r * kPRowBytes;
+    const uint32_t swz = (static_cast<uint32_t>(r) >> 2) & 1u;   // 32-byte swizzle of this row
 
     for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      ok = mbar_wait(&s.bar_s_full[sb], (j >> 1) & 1, abort_flag, p.status, kStatusTimeoutS | 8 | sb);
+      ok = mbar_wait(&s.bar_s_full, j & 1, abort_flag, p.status, kStatusTimeoutS | 8);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -293,14 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t raw[32];
 #pragma unroll
         for (int cc = 0; cc < kBN / 32; ++cc) {
-          tmem_ld32(tmem + lane_addr + (sb ? kColS1 : kColS0) + cc * 32, raw);
+          tmem_ld32(tmem + lane_addr + kColS + cc * 32, raw);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(raw[i]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&s.bar_s_empty[sb]);
+      mbar_arrive(&s.bar_s_empty);
 
       // masking: keys beyond N, and keys after the query row when causal
       const int key0 = j * kBN;
@@ -313,41 +327,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float bmax[kBN / 32];
 #pragma unroll
-      for (int bb = 0; bb < kBN / 32; ++bb) {
-        float mx = sv[bb * 32];
-#pragma unroll
-        for (int i = 1; i < 32; ++i) mx = fmaxf(mx, sv[bb * 32 + i]);
-        bmax[bb] = mx;
-      }
-      float tmax = bmax[0];
-#pragma unroll
-      for (int bb = 1; bb < kBN / 32; ++bb) tmax = fmaxf(tmax, bmax[bb]);
-      const float m_new = fmaxf(m, tmax);
+      for (int bb = 0; bb < kBN / 32; ++bb) bmax[bb] = block_max32(sv + bb * 32);
+      const float m_new = fmaxf(m, fmaxf(bmax[0], bmax[1]));
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
 
-      uint32_t words[kBN / 8];          // 16 words = 64 bytes of codes for this row
-      uint32_t sbytes = 0;
-      float tile_sum = 0.f;
+      // per 32-key block: amax from the exact difference (1 for the block that holds the max),
+      // its E8M0 byte, and the exponent bias of y = P~ / 2^e = 2^(S c - m c - e)
+      uint32_t byte[kBN / 32];
+      float nb[kBN / 32];
 #pragma unroll
       for (int bb = 0; bb < kBN / 32; ++bb) {
         const float amax = ex2_approx((bmax[bb] - m_use) * c);     // 0 for an all-masked block
-        const uint32_t byte = e8m0_scale_byte(amax, p.mode);
-        sbytes |= byte << (8 * bb);
-        const float neg_e = static_cast<float>(127 - static_cast<int>(byte));
-        float y[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] = ex2_approx_ftz(fmaf(sv[bb * 32 + i] - m_use, c, neg_e));
-#pragma unroll
-        for (int w = 0; w < 4; ++w) words[bb * 4 + w] = cvt_e2m1x8(y + 8 * w);
-        if (!p.pnq) {   // conventional row sum of the unquantized exponentials
-          float bsum = 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) bsum += y[i];
-          tile_sum = fmaf(bsum, pow2_from_byte(byte), tile_sum);
-        }
+        byte[bb] = e8m0_scale_byte(amax, p.mode);
+        nb[bb] = fmaf(-m_use, c, static_cast<float>(127 - static_cast<int>(byte[bb])));
       }
-      l = fmaf(alpha, l, tile_sum);      // (with PNQ the row sum accumulates in TMEM instead)
+      const uint32_t sbytes = byte[0] | (byte[1] << 8);
+      // y for the whole tile (one FFMA + one ex2 per element), then the E2M1 codes
+      float y[kBN];
+#pragma unroll
+      for (int i = 0; i < kBN; ++i) y[i] = ex2_approx_ftz(fmaf(sv[i], c, nb[i / 32]));
+      uint32_t words[kBN / 8];          // 8 words = 32 bytes of codes for this row
+#pragma unroll
+      for (int w = 0; w < kBN / 8; ++w) words[w] = cvt_e2m1x8(y + 8 * w);
+      if (!PNQ) {   // conventional row sum of the unquantized exponentials
+        float tile_sum = 0.f;
+#pragma unroll
+        for (int bb = 0; bb < kBN / 32; ++bb) {
+          float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            b0 += y[bb * 32 + i];
+            b1 += y[bb * 32 + i + 1];
+          }
+          tile_sum = fmaf(b0 + b1, pow2_from_byte(byte[bb]), tile_sum);
+        }
+        l = fmaf(alpha, l, tile_sum);
+      }
 
       // P~ buffer and O are free once the previous P~V product has completed
       if (j > 0) {
@@ -357,34 +373,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const uint4 v4 = make_uint4(words[ch * 4], words[ch * 4 + 1], words[ch * 4 + 2], words[ch * 4 + 3]);
-        *reinterpret_cast<uint4*>(p_row + ((ch ^ swz) << 4)) = v4;
+      for (int bb = 0; bb < kBN / 32; ++bb) {
+        const uint4 v4 = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
+        *reinterpret_cast<uint4*>(p_row + ((bb ^ swz) << 4)) = v4;
       }
-      *reinterpret_cast<uint32_t*>(s.psf + ((r & 31) * 16 + (r >> 5) * 4)) = sbytes;
+      *reinterpret_cast<uint16_t*>(s.psf + ((r & 31) * 16 + (r >> 5) * 4)) = static_cast<uint16_t>(sbytes);
       if (dbg) {
         uint4* dc = reinterpret_cast<uint4*>(p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) +
-                                             j * (kBN / 2));
+                                             j * kPRowBytes);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          dc[ch] = make_uint4(words[ch * 4], words[ch * 4 + 1], words[ch * 4 + 2], words[ch * 4 + 3]);
-        *reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 32) +
-                                     j * 4) = sbytes;
+        for (int bb = 0; bb < kBN / 32; ++bb)
+          dc[bb] = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
+        *reinterpret_cast<uint16_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 32) +
+                                     j * 2) = static_cast<uint16_t>(sbytes);
       }
       fence_proxy_async_smem();
 
-      // history rescale of O (only when some row of this warp saw its max move)
+      // history rescale of O and L (only when some row of this warp saw its max move)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t raw[32];
-          tmem_ld32(tmem + lane_addr + kColO + cc * 32, raw);
+          const uint32_t col = tmem + lane_addr + kColO + cc * 32;
+          tmem_ld32(col, raw);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-          tmem_st32(tmem + lane_addr + kColO + cc * 32, raw);
+          tmem_st32(col, raw);
         }
-        if (p.pnq) {
+        if (PNQ) {
           const uint32_t lv = tmem_ld1(tmem + lane_addr + kColL);
           tc_wait_ld();
           tmem_st1(tmem + lane_addr + kColL, __float_as_uint(__uint_as_float(lv) * alpha));
@@ -403,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      if (p.pnq) {
+      if (PNQ) {
         l = __uint_as_float(tmem_ld1(tmem + lane_addr + kColL));
         tc_wait_ld();
       }
@@ -450,22 +467,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool PNQ>
 static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * (p.Npad / kBM);
-  mxattn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PNQ><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const AttnParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, p, stream);
-  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, p, stream);
+  if (d == 128) return p.pnq ? launch_d<128, true>(tmQ, tmK, tmV, p, stream)
+                             : launch_d<128, false>(tmQ, tmK, tmV, p, stream);
+  if (d == 64) return p.pnq ? launch_d<64, true>(tmQ, tmK, tmV, p, stream)
+                            : launch_d<64, false>(tmQ, tmK, tmV, p, stream);
   return cudaErrorInvalidValue;
 }
 

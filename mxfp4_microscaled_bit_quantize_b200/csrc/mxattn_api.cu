@@ -130,8 +130,9 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!make_map(&tq, w + L.qc, d / 2, static_cast<uint64_t>(B) * Hq * L.npad, d / 2, kTile, qk_swz) ||
-      !make_map(&tk, w + L.kc, d / 2, static_cast<uint64_t>(B) * Hkv * L.npad, d / 2, kTile, qk_swz) ||
-      !make_map(&tv, w + L.vc, L.npad / 2, static_cast<uint64_t>(B) * Hkv * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
+      !make_map(&tk, w + L.kc, d / 2, static_cast<uint64_t>(B) * Hkv * L.npad, d / 2, kKvTile, qk_swz) ||
+      !make_map(&tv, w + L.vc, L.npad / 2, static_cast<uint64_t>(B) * Hkv * d, kKvTile / 2, d,
+                CU_TENSOR_MAP_SWIZZLE_32B))
     return MXATTN_ERR_CUDA;
   AttnParams p{};
   p.qsf = w + L.qs;
@@ -178,7 +179,7 @@ mxattn_status check_forward_args(const void* q, const void* k, const void* v, co
 
 extern "C" {
 
-int mxattn_version(void) { return 100; }
+int mxattn_version(void) { return 101; }
 
 const char* mxattn_status_string(int status) {
   switch (status) {

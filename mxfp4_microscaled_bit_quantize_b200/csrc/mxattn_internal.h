@@ -7,6 +7,10 @@
 
 namespace mxattn {
 
+// Keys per KV tile of the attention kernel: P~ is quantized with the running max in force at
+// each tile, so this width is part of what the kernel computes (MXATTN_KV_TILE in mxattn.h).
+constexpr int kKvTile = 64;
+
 enum SfLayout : int { kSfRowMajor = 0, kSfAtom = 1 };
 
 // Blocks of 32 along the contiguous axis of `heads` matrices of [rows, cols] bf16. Rows in

@@ -53,6 +53,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed sleeps in hardware
+// until the phase completes or about `hint_ns` pass, instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 50000;   // per sleep; the 2 s bound is checked between sleeps
+
 // Wait until the barrier's phase with the given parity has completed. Gives up (returning
 // false) when another thread of the CTA raised the abort flag or after kWaitTimeoutNs; in the
 // timeout case the status word receives `code` (first writer wins) and the abort flag is set.
@@ -60,15 +76,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           unsigned int* status, unsigned int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        atomicCAS(status, 0u, code);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      atomicCAS(status, 0u, code);
+      return false;
     }
   }
 }
@@ -216,6 +230,13 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, uint32_t a_sf_id, 
          (a_sf_id << 29);
 }
 
+// max(a, b, c) in one instruction (three-input form, sm_100+).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // ------------------------------------------------------------------ E2M1 conversion
 
 // Two fp32 values -> one byte of E2M1 codes (round to nearest even, saturating at 6);
@@ -250,25 +271,16 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
 //   OCP (mode 0): e = floor(log2 amax) - 2.
 //   UOS (mode 1): the smallest e with amax / 2^e <= 7.25, i.e. the OCP exponent plus one when
 //                 the significand of amax exceeds 1.8125 (7.25 / 4).
-// amax == 0 gives byte 0; the result is clamped to [0, 254].
+// amax == 0 gives byte 0; the result is clamped to [0, 254]. Branch-free: a subnormal amax is
+// first scaled by 2^64 (exact) so that its exponent and significand can be read off the bits.
 __device__ __forceinline__ uint32_t e8m0_scale_byte(float amax, int mode) {
-  const uint32_t bits = __float_as_uint(amax);
-  if (bits == 0u) return 0u;
-  int e0;            // floor(log2 amax)
-  uint32_t mant;     // 23-bit fraction of the normalised significand
-  const uint32_t bexp = bits >> 23;
-  if (bexp != 0u) {
-    e0 = static_cast<int>(bexp) - 127;
-    mant = bits & 0x7FFFFFu;
-  } else {           // subnormal: normalise the fraction
-    const int lz = __clz(bits) - 8;           // leading zeros inside the 24-bit significand field
-    e0 = -126 - lz;
-    mant = (bits << lz) & 0x7FFFFFu;
-  }
-  int e = e0 - 2;
-  if (mode == 1 && mant > 0x680000u) e += 1;  // significand > 1.8125
+  const bool sub = __float_as_uint(amax) < 0x00800000u;           // subnormal or zero
+  const uint32_t bits = __float_as_uint(sub ? amax * 18446744073709551616.0f : amax);
+  const int e0 = static_cast<int>(bits >> 23) - (sub ? 191 : 127);  // floor(log2 amax)
+  const uint32_t mant = bits & 0x7FFFFFu;
+  int e = e0 - 2 + ((mode == 1 && mant > 0x680000u) ? 1 : 0);
   e = max(-127, min(127, e));
-  return static_cast<uint32_t>(e + 127);
+  return amax == 0.0f ? 0u : static_cast<uint32_t>(e + 127);
 }
 
 // 2^-e as an fp32 (normal for every e in [-126, 127]; e = -127 gives 2^127).

@@ -49,7 +49,7 @@ import numpy as np
 
 from . import mxfp4 as mx
 
-KV_TILE = 128
+KV_TILE = 64          # the library's documented tile width (MXATTN_KV_TILE)
 
 
 def dequantized_qkv(q, k, v, mode: int):

@@ -108,3 +108,12 @@ def test_debug_argument_checks(lib):
     r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
                                  0, 10, 5, FAKE, FAKE)   # empty row range
     assert r == INVALID
+
+
+def test_kv_tile_constant_agrees():
+    """P~ codes depend on the online-softmax tile width; the binding and the oracle's default
+    must use the width the library declares."""
+    from mxfp4_microscaled_bit_quantize_b200 import api
+    from oracle import attention as oa
+    m = re.search(r"#define\s+MXATTN_KV_TILE\s+(\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == api.KV_TILE == oa.KV_TILE
