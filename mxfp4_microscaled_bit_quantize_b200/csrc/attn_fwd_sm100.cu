@@ -67,20 +67,22 @@ struct __align__(1024) Smem {
   uint8_t q[Cfg<D>::kQTileBytes];
   uint8_t k[Cfg<D>::kStages][Cfg<D>::kKTileBytes];
   uint8_t v[Cfg<D>::kStages][Cfg<D>::kVTileBytes];
-  uint8_t p[kBM * kPRowBytes];
+  uint8_t p[2][kBM * kPRowBytes];         // P~ codes, double-buffered by tile parity
   uint8_t ones[kOnesRows * kPRowBytes];
   uint8_t qsf[512];
   uint8_t ksf[Cfg<D>::kStages][512];
   uint8_t vsf[Cfg<D>::kStages][512];
-  uint8_t psf[512];
+  uint8_t psf[2][512];
   uint8_t onesf[512];
   uint64_t bar_q;
   uint64_t bar_kv_full[Cfg<D>::kStages];
   uint64_t bar_kv_empty[Cfg<D>::kStages];
   uint64_t bar_s_full;
   uint64_t bar_s_empty;
-  uint64_t bar_p_full;
-  uint64_t bar_pv_done;
+  // P~ buffer b written by all 128 rows (tiles of parity b). One barrier per buffer: a fast
+  // softmax warp may arrive for tile j+1 before a slow one has arrived for tile j.
+  uint64_t bar_p_full[2];
+  uint64_t bar_pv_done[2];                 // completions of PV of even / odd tiles
   uint64_t bar_drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -129,7 +131,7 @@ __device__ __forceinline__ float block_max32(const float* v) {
   return fmaxf(fmax3(a0, a1, a2), a3);
 }
 
-template <int D, bool PNQ>
+template <int D, bool PNQ, bool DBG>
 __global__ void __launch_bounds__(kThreads, 2)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -164,8 +166,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(&s.bar_s_full, 1);
     mbar_init(&s.bar_s_empty, kBM);
-    mbar_init(&s.bar_p_full, kBM);
-    mbar_init(&s.bar_pv_done, 1);
+    mbar_init(&s.bar_p_full[0], kBM);
+    mbar_init(&s.bar_p_full[1], kBM);
+    mbar_init(&s.bar_pv_done[0], 1);
+    mbar_init(&s.bar_pv_done[1], 1);
     mbar_init(&s.bar_drain, 1);
     s.abort_flag = 0;
     fence_mbar_init();
@@ -182,21 +186,26 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 0) {
     // ============================ TMA producer ============================
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform operands); one elected lane issues the copies.
+    const bool leader = elect_one_sync();
+    if (leader) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&s.bar_q, C::kQTileBytes + 512);
       tma_load_2d(s.q, &tmQ, &s.bar_q, 0, bh_q * p.Npad + qt * kBM);
       bulk_load(s.qsf, p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt) * 512, 512, &s.bar_q);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % NS;
-        if (j >= NS) {
-          if (!mbar_wait(&s.bar_kv_empty[st], ((j / NS) & 1) ^ 1, abort_flag, p.status,
-                         kStatusTimeoutEmpty | st))
-            break;
-        }
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j % NS;
+      if (j >= NS) {
+        bool ok = mbar_wait(&s.bar_kv_empty[st], ((j / NS) & 1) ^ 1, abort_flag, p.status,
+                            kStatusTimeoutEmpty | st);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      if (leader) {
         mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + 1024);
         tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.Npad + j * kBN);
         tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
@@ -204,46 +213,57 @@ __global__ void __launch_bounds__(kThreads, 2)
         const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;
         bulk_load(s.ksf[st], p.ksf + atom, 512, &s.bar_kv_full[st]);
         bulk_load(s.vsf[st], p.vsf + atom, 512, &s.bar_kv_full[st]);
-        issued = j + 1;
       }
-      if (*abort_flag) {
-        // let every copy this thread started land before the CTA can exit
-        drain_wait(&s.bar_q, 0);
-        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-          drain_wait(&s.bar_kv_full[j % NS], (j / NS) & 1);
-      }
+      __syncwarp();
+      issued = j + 1;
     }
+    if (*abort_flag && leader) {
+      // let every copy this warp started land before the CTA can exit
+      drain_wait(&s.bar_q, 0);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        drain_wait(&s.bar_kv_full[j % NS], (j / NS) & 1);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
-      const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
-      auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
-      if (PNQ) {
-        // ones operand (row 0 = code 1.0 for every key, rows 1..15 = 0) with unit scales
-        uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
-        for (int i = 0; i < kOnesRows * kPRowBytes / 4; ++i) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
-        uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
-        for (int i = 0; i < 512 / 4; ++i) sw[i] = 0x7F7F7F7Fu;
-        fence_proxy_async_smem();
-      }
-      bool ok = mbar_wait(&s.bar_q, 0, abort_flag, p.status, kStatusTimeoutQ);
-      if (ok) {
-        tc_fence_after();
+    // The whole warp runs the loop (warp-uniform descriptors); one elected lane issues every
+    // tcgen05 operation and commit, so completion tracking stays with that thread.
+    const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
+    auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
+    if (PNQ) {
+      // ones operand (row 0 = code 1.0 for every key, rows 1..15 = 0) with unit scales
+      uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
+      for (int i = lane; i < kOnesRows * kPRowBytes / 4; i += 32) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
+      uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
+      for (int i = lane; i < 512 / 4; i += 32) sw[i] = 0x7F7F7F7Fu;
+      fence_proxy_async_smem();
+    }
+    __syncwarp();
+    const bool leader = elect_one_sync();
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_q, 0, abort_flag, p.status, kStatusTimeoutQ));
+    if (ok) {
+      tc_fence_after();
+      if (leader) {
         tc_cp_sf(tmem + kColSfQ, sf_desc(s.qsf));
         if (PNQ) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
       }
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % NS;
-        if (!mbar_wait(&s.bar_kv_full[st], (j / NS) & 1, abort_flag, p.status, kStatusTimeoutKV | st))
-          return false;
-        // S is single-buffered: the previous tile must be in the softmax registers
-        if (j >= 1 && !mbar_wait(&s.bar_s_empty, (j - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
-          return false;
-        tc_fence_after();
+      __syncwarp();
+    }
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_kv_full[st], (j / NS) & 1, abort_flag, p.status,
+                                             kStatusTimeoutKV | st)))
+        return false;
+      // S is single-buffered: the previous tile must be in the softmax registers
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&s.bar_s_empty, (j - 1) & 1, abort_flag, p.status,
+                                                       kStatusTimeoutS)))
+        return false;
+      tc_fence_after();
+      const uint32_t qa = smem_u32(s.q), ka = smem_u32(s.k[st]);
+      // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
+      const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
+      if (leader) {
         tc_cp_sf(tmem + kColSfK, sf_desc(s.ksf[st]));
-        const uint32_t qa = smem_u32(s.q), ka = smem_u32(s.k[st]);
-        // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
-        const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
           const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
@@ -251,17 +271,21 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ, sfk, kk > 0);
         }
         tc_commit(&s.bar_s_full);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % NS;
-        if (!mbar_wait(&s.bar_p_full, j & 1, abort_flag, p.status, kStatusTimeoutP)) return false;
-        tc_fence_after();
-        tc_cp_sf(tmem + kColSfP, sf_desc(s.psf));
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int j) -> bool {
+      const int st = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_p_full[j & 1], (j >> 1) & 1, abort_flag, p.status, kStatusTimeoutP)))
+        return false;
+      tc_fence_after();
+      const uint32_t pa = smem_u32(s.p[j & 1]), va = smem_u32(s.v[st]);
+      const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
+      const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
+      if (leader) {
+        tc_cp_sf(tmem + kColSfP, sf_desc(s.psf[j & 1]));
         tc_cp_sf(tmem + kColSfV, sf_desc(s.vsf[st]));
-        const uint32_t pa = smem_u32(s.p), va = smem_u32(s.v[st]);
-        const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
-        const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
         // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
         tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), tmem + kColSfP, tmem + kColSfV,
                     j > 0 ? 1u : 0u);
@@ -270,19 +294,23 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), tmem + kColSfP, tmem + kColSf1,
                       j > 0 ? 1u : 0u);
         }
-        tc_commit(&s.bar_pv_done);
+        tc_commit(&s.bar_pv_done[j & 1]);
         tc_commit(&s.bar_kv_empty[st]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
       }
-      // every MMA / copy issued above must complete before TMEM is released
+      __syncwarp();
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      if (j + 1 < n_kv) ok = issue_s(j + 1);
+      if (ok) ok = issue_pv(j);
+    }
+    // every MMA / copy issued above must complete before TMEM is released
+    if (leader) {
       tc_commit(&s.bar_drain);
       drain_wait(&s.bar_drain, 0);
     }
+    __syncwarp();
   } else {
     // ============================ softmax warpgroup ============================
     const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
@@ -293,8 +321,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m = -INFINITY;      // running max of the raw scores S
     float l = 0.f;            // running row sum (pnq = 0)
     bool ok = true;
-    const bool dbg = p.dbg_codes != nullptr && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
-    uint8_t* p_row = s.p + r * kPRowBytes;
+    const bool dbg = DBG && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
+    const uint32_t p_row_off = r * kPRowBytes;
+    const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
     const uint32_t swz = (static_cast<uint32_t>(r) >> 2) & 1u;   // 32-byte swizzle of this row
 
     for (int j = 0; j < n_kv; ++j) {
@@ -365,20 +394,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         l = fmaf(alpha, l, tile_sum);
       }
 
-      // P~ buffer and O are free once the previous P~V product has completed
-      if (j > 0) {
-        ok = mbar_wait(&s.bar_pv_done, (j - 1) & 1, abort_flag, p.status, kStatusTimeoutPV);
+      // P~ buffer j&1 is free once the product of tile j-2 (its last reader) has completed
+      const int pb = j & 1;
+      if (j >= 2) {
+        ok = mbar_wait(&s.bar_pv_done[pb], ((j >> 1) - 1) & 1, abort_flag, p.status, kStatusTimeoutPV);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        tc_fence_after();
       }
+      uint8_t* p_row = s.p[pb] + p_row_off;
 #pragma unroll
       for (int bb = 0; bb < kBN / 32; ++bb) {
         const uint4 v4 = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
         *reinterpret_cast<uint4*>(p_row + ((bb ^ swz) << 4)) = v4;
       }
-      *reinterpret_cast<uint16_t*>(s.psf + ((r & 31) * 16 + (r >> 5) * 4)) = static_cast<uint16_t>(sbytes);
-      if (dbg) {
+      *reinterpret_cast<uint16_t*>(s.psf[pb] + psf_off) = static_cast<uint16_t>(sbytes);
+      if (DBG && dbg) {
         uint4* dc = reinterpret_cast<uint4*>(p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) +
                                              j * kPRowBytes);
 #pragma unroll
@@ -389,8 +419,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       fence_proxy_async_smem();
 
-      // history rescale of O and L (only when some row of this warp saw its max move)
+      // history rescale of O and L (only when some row of this warp saw its max move); O may only
+      // be touched once the product of tile j-1 has landed in it
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        ok = mbar_wait(&s.bar_pv_done[pb ^ 1], ((j - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t raw[32];
@@ -409,13 +444,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&s.bar_p_full);
+      mbar_arrive(&s.bar_p_full[pb]);
       m = m_new;
     }
 
-    // ---- epilogue: out = O / l
+    // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
     if (ok) {
-      ok = mbar_wait(&s.bar_pv_done, (n_kv - 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 1);
+      ok = mbar_wait(&s.bar_pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
+                     kStatusTimeoutPV | 1);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -467,24 +503,32 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D, bool PNQ>
-static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+template <int D, bool PNQ, bool DBG>
+static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ, DBG>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * (p.Npad / kBM);
-  mxattn_fwd_kernel<D, PNQ><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PNQ, DBG><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const AttnParams& p, cudaStream_t stream) {
+  const bool dbg = p.dbg_codes != nullptr;
+  if (p.pnq) return dbg ? launch_k<D, true, true>(tmQ, tmK, tmV, p, stream)
+                        : launch_k<D, true, false>(tmQ, tmK, tmV, p, stream);
+  return dbg ? launch_k<D, false, true>(tmQ, tmK, tmV, p, stream)
+             : launch_k<D, false, false>(tmQ, tmK, tmV, p, stream);
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const AttnParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return p.pnq ? launch_d<128, true>(tmQ, tmK, tmV, p, stream)
-                             : launch_d<128, false>(tmQ, tmK, tmV, p, stream);
-  if (d == 64) return p.pnq ? launch_d<64, true>(tmQ, tmK, tmV, p, stream)
-                            : launch_d<64, false>(tmQ, tmK, tmV, p, stream);
+  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, p, stream);
+  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, p, stream);
   return cudaErrorInvalidValue;
 }
 
