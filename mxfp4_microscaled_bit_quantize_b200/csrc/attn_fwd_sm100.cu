@@ -29,7 +29,7 @@
 //              quantizes it in registers, writes codes (32B-swizzled, the MMA operand layout)
 //              and scale bytes to shared memory, rescales O and L in TMEM when the max moves,
 //              and finally normalises and stores the output.
-// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..231.
+// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..235.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -44,7 +44,13 @@ constexpr int kBN = kKvTile;      // keys per KV tile (64)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 64, kColL = 192;
-constexpr uint32_t kColSfQ = 208, kColSfK = 212, kColSfV = 216, kColSfP = 220, kColSf1 = 224;
+constexpr uint32_t kColSfQ = 208, kColSfK = 212, kColSf1 = 216;
+// P~ scale atoms alternate between two column sets by tile parity, V scale atoms (one per pair of
+// 64-key tiles) by pair parity: tcgen05.cp into columns an earlier MMA still reads is not ordered
+// behind that MMA, and the product of tile j may still run when the scales of tile j+1 are
+// copied. The set written for tile j+1 was last read by a product no later than that of tile
+// j-1, which the softmax has seen complete before it hands over tile j+1.
+constexpr uint32_t kColSfV = 220, kColSfP = 228;   // + 4 * set
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
 constexpr int kPRowBytes = kBN / 2;                  // 32 bytes of codes per P~ row
 constexpr size_t kMinSmem = 80 * 1024;               // at most two CTAs per SM (TMEM halves)
@@ -206,13 +212,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (leader) {
-        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + 1024);
+        // scale atoms cover 128 keys: tiles 2t and 2t+1 share atom t, loaded with the even tile
+        const bool atoms = (j & 1) == 0;
+        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + (atoms ? 1024 : 0));
         tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.Npad + j * kBN);
         tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
-        // scale atoms cover 128 keys: tiles 2t and 2t+1 share atom t
-        const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;
-        bulk_load(s.ksf[st], p.ksf + atom, 512, &s.bar_kv_full[st]);
-        bulk_load(s.vsf[st], p.vsf + atom, 512, &s.bar_kv_full[st]);
+        if (atoms) {
+          const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;
+          bulk_load(s.ksf[st], p.ksf + atom, 512, &s.bar_kv_full[st]);
+          bulk_load(s.vsf[st], p.vsf + atom, 512, &s.bar_kv_full[st]);
+        }
       }
       __syncwarp();
       issued = j + 1;
@@ -263,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
       const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
       if (leader) {
-        tc_cp_sf(tmem + kColSfK, sf_desc(s.ksf[st]));
+        // the even tile brings the K atom of the pair; S of the previous pair has completed
+        if ((j & 1) == 0) tc_cp_sf(tmem + kColSfK, sf_desc(s.ksf[st]));
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
           const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
@@ -284,14 +294,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
       const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
       if (leader) {
-        tc_cp_sf(tmem + kColSfP, sf_desc(s.psf[j & 1]));
-        tc_cp_sf(tmem + kColSfV, sf_desc(s.vsf[st]));
+        const uint32_t sfp = tmem + kColSfP + 4 * (j & 1), sfv = tmem + kColSfV + 4 * ((j >> 1) & 1);
+        tc_cp_sf(sfp, sf_desc(s.psf[j & 1]));
+        if ((j & 1) == 0) tc_cp_sf(sfv, sf_desc(s.vsf[st]));   // the V atom of the tile pair
         // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
-        tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), tmem + kColSfP, tmem + kColSfV,
+        tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), sfp, sfv,
                     j > 0 ? 1u : 0u);
         if (PNQ) {
           const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
-          tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), tmem + kColSfP, tmem + kColSf1,
+          tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), sfp, tmem + kColSf1,
                       j > 0 ? 1u : 0u);
         }
         tc_commit(&s.bar_pv_done[j & 1]);
@@ -333,13 +344,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       float sv[kBN];
       {
-        uint32_t raw[32];
+        uint32_t raw0[32], raw1[32];
+        tmem_ld32(tmem + lane_addr + kColS, raw0);
+        tmem_ld32(tmem + lane_addr + kColS + 32, raw1);
+        tc_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          tmem_ld32(tmem + lane_addr + kColS + cc * 32, raw);
-          tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(raw[i]);
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = __uint_as_float(raw0[i]);
+          sv[32 + i] = __uint_as_float(raw1[i]);
         }
       }
       tc_fence_before();
@@ -427,14 +439,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t raw[32];
+        for (int cc = 0; cc < D / 32; cc += 2) {   // 64 columns per round trip
+          uint32_t raw0[32], raw1[32];
           const uint32_t col = tmem + lane_addr + kColO + cc * 32;
-          tmem_ld32(col, raw);
+          tmem_ld32(col, raw0);
+          tmem_ld32(col + 32, raw1);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-          tmem_st32(col, raw);
+          for (int i = 0; i < 32; ++i) {
+            raw0[i] = __float_as_uint(__uint_as_float(raw0[i]) * alpha);
+            raw1[i] = __float_as_uint(__uint_as_float(raw1[i]) * alpha);
+          }
+          tmem_st32(col, raw0);
+          tmem_st32(col + 32, raw1);
         }
         if (PNQ) {
           const uint32_t lv = tmem_ld1(tmem + lane_addr + kColL);
