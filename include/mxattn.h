@@ -103,6 +103,27 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mxattn_forward_quantized -- the attention kernel alone, on Q, K and V already in MXFP4 (MXAttention
+ * abstract: MXFP4 operands for Q K^T and P~ V; P~ is quantized inside, with PNQ when pnq = 1).
+ * The operands are in the canonical layout that mxattn_quantize writes:
+ *   qc  : codes  [B, Hq,  N, d/2]   (mxattn_quantize of q, transpose = 0), 16-byte aligned
+ *   qs  : scales [B, Hq,  N, d/32]  E8M0 bytes
+ *   kc  : codes  [B, Hkv, N, d/2],  ks: scales [B, Hkv, N, d/32]
+ *   vtc : codes  [B, Hkv, d, ceil(N/32)*16]  (mxattn_quantize of v with transpose = 1: blocks of
+ *         32 keys, keys past N encoded as zero), 16-byte aligned
+ *   vts : scales [B, Hkv, d, ceil(N/32)]
+ *   p_scale_mode: the scale rule for P~ (the caller chose the rule of Q, K, V when quantizing).
+ * All other arguments as mxattn_forward; the workspace (mxattn_forward_workspace_size bytes)
+ * receives the scales in the tensor-core layout and the status word; the codes are read in place
+ * and must stay unchanged until the call has completed on the stream. Errors: null or misaligned
+ * pointers -> MXATTN_ERR_INVALID_ARG; shapes as mxattn_forward.
+ */
+mxattn_status mxattn_forward_quantized(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                                       const uint8_t* vtc, const uint8_t* vts, void* out, int B, int Hq, int Hkv,
+                                       int N, int d, int causal, int p_scale_mode, int pnq, int out_dtype,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The two halves of mxattn_forward, for callers that time or reuse them separately:
  *   mxattn_forward_prepare quantizes q, k, v into the workspace;
  *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same

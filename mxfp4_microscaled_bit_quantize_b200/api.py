@@ -107,6 +107,38 @@ def mxattn_forward(q, k, v, causal: bool = False, scale_mode: int = SCALE_UOS, p
     return out
 
 
+def mxattn_forward_quantized(qc, qs, kc, ks, vtc, vts, N: int, d: int, causal: bool = False,
+                             p_scale_mode: int = SCALE_UOS, pnq: bool = True, out_dtype=torch.float32,
+                             workspace: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """The attention kernel on operands already in MXFP4 (the layout mxattn_quantize writes):
+    qc [B,Hq,N,d/2] / qs [B,Hq,N,d/32], kc / ks [B,Hkv,N,..], vtc [B,Hkv,d,ceil(N/32)*16] /
+    vts [B,Hkv,d,ceil(N/32)], all uint8 CUDA tensors. Returns out [B,Hq,N,d]."""
+    for t, n in ((qc, "qc"), (qs, "qs"), (kc, "kc"), (ks, "ks"), (vtc, "vtc"), (vts, "vts")):
+        _need(t, n, torch.uint8)
+    nb = -(-N // 32)
+    B, Hq = int(qc.shape[0]), int(qc.shape[1])
+    Hkv = int(kc.shape[1])
+    shapes = {"qc": (B, Hq, N, d // 2), "qs": (B, Hq, N, d // 32), "kc": (B, Hkv, N, d // 2),
+              "ks": (B, Hkv, N, d // 32), "vtc": (B, Hkv, d, nb * 16), "vts": (B, Hkv, d, nb)}
+    for t, n in ((qc, "qc"), (qs, "qs"), (kc, "kc"), (ks, "ks"), (vtc, "vtc"), (vts, "vts")):
+        if tuple(t.shape) != shapes[n]:
+            raise ValueError(f"{n} must have shape {shapes[n]}, got {tuple(t.shape)}")
+    dt = torch.float32 if out_dtype in (OUT_F32, torch.float32) else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=dt, device=qc.device)
+    else:
+        _need(out, "out", dt)
+    od = OUT_F32 if dt == torch.float32 else OUT_BF16
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, N, d, qc.device)
+    st = _lib.load().mxattn_forward_quantized(qc.data_ptr(), qs.data_ptr(), kc.data_ptr(), ks.data_ptr(),
+                                              vtc.data_ptr(), vts.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                                              int(bool(causal)), int(p_scale_mode), int(bool(pnq)), od,
+                                              workspace.data_ptr(), workspace.numel(), _stream(qc.device))
+    _lib.check(st, "mxattn_forward_quantized")
+    return out
+
+
 def mxattn_forward_prepare(q, k, v, scale_mode: int, workspace: torch.Tensor) -> None:
     B, Hq, Hkv, N, d = _shapes(q, k, v)
     st = _lib.load().mxattn_forward_prepare(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d,

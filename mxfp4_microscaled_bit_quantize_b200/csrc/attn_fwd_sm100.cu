@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&s.bar_q, C::kQTileBytes + 512);
-      tma_load_2d(s.q, &tmQ, &s.bar_q, 0, bh_q * p.Npad + qt * kBM);
+      tma_load_2d(s.q, &tmQ, &s.bar_q, 0, bh_q * p.rows_per_head + qt * kBM);
       bulk_load(s.qsf, p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt) * 512, 512, &s.bar_q);
     }
     __syncwarp();
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // scale atoms cover 128 keys: tiles 2t and 2t+1 share atom t, loaded with the even tile
         const bool atoms = (j & 1) == 0;
         mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + (atoms ? 1024 : 0));
-        tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.Npad + j * kBN);
+        tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.rows_per_head + j * kBN);
         tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
         if (atoms) {
           const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;

@@ -123,15 +123,31 @@ mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, i
   return MXATTN_OK;
 }
 
+// Where the attention kernel reads its FP4 codes: the workspace (rows padded to Npad, V^T rows of
+// Npad/2 bytes) or caller tensors in the canonical layout (N rows per head, V^T rows of
+// ceil(N/32)*16 bytes). Rows and keys past N are never used: padded query rows are not stored,
+// keys >= N are masked, and the tensor maps zero-fill reads past the last row or column.
+struct CodeSources {
+  const uint8_t *qc, *kc, *vc;
+  int rows_per_head;
+  uint64_t v_row_bytes;
+};
+
+CodeSources workspace_codes(void* ws, const WsLayout& L) {
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  return CodeSources{w + L.qc, w + L.kc, w + L.vc, L.npad, static_cast<uint64_t>(L.npad) / 2};
+}
+
 mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int causal, int scale_mode, int pnq,
-                          int out_dtype, void* ws, cudaStream_t st, const WsLayout& L, int dbg_bh, int dbg_r0,
-                          int dbg_r1, uint8_t* p_codes, uint8_t* p_scales) {
+                          int out_dtype, void* ws, cudaStream_t st, const WsLayout& L, const CodeSources& src,
+                          int dbg_bh, int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!make_map(&tq, w + L.qc, d / 2, static_cast<uint64_t>(B) * Hq * L.npad, d / 2, kTile, qk_swz) ||
-      !make_map(&tk, w + L.kc, d / 2, static_cast<uint64_t>(B) * Hkv * L.npad, d / 2, kKvTile, qk_swz) ||
-      !make_map(&tv, w + L.vc, L.npad / 2, static_cast<uint64_t>(B) * Hkv * d, kKvTile / 2, d,
+  const uint64_t rph = static_cast<uint64_t>(src.rows_per_head);
+  if (!make_map(&tq, src.qc, d / 2, static_cast<uint64_t>(B) * Hq * rph, d / 2, kTile, qk_swz) ||
+      !make_map(&tk, src.kc, d / 2, static_cast<uint64_t>(B) * Hkv * rph, d / 2, kKvTile, qk_swz) ||
+      !make_map(&tv, src.vc, src.v_row_bytes, static_cast<uint64_t>(B) * Hkv * d, kKvTile / 2, d,
                 CU_TENSOR_MAP_SWIZZLE_32B))
     return MXATTN_ERR_CUDA;
   AttnParams p{};
@@ -145,6 +161,7 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   p.Hkv = Hkv;
   p.N = N;
   p.Npad = L.npad;
+  p.rows_per_head = src.rows_per_head;
   p.causal = causal ? 1 : 0;
   p.mode = scale_mode;
   p.pnq = pnq ? 1 : 0;
@@ -265,7 +282,35 @@ mxattn_status mxattn_forward_attend(void* out, int B, int Hq, int Hkv, int N, in
                                        workspace, workspace_bytes, &L);
   if (s != MXATTN_OK) return s;
   return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace,
-                     static_cast<cudaStream_t>(stream), L, -1, 0, 0, nullptr, nullptr);
+                     static_cast<cudaStream_t>(stream), L, workspace_codes(workspace, L), -1, 0, 0, nullptr,
+                     nullptr);
+}
+
+mxattn_status mxattn_forward_quantized(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                                       const uint8_t* vtc, const uint8_t* vts, void* out, int B, int Hq, int Hkv,
+                                       int N, int d, int causal, int p_scale_mode, int pnq, int out_dtype,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!qc || !qs || !kc || !ks || !vtc || !vts || !out) return MXATTN_ERR_INVALID_ARG;
+  if (!aligned(qc, 16) || !aligned(kc, 16) || !aligned(vtc, 16)) return MXATTN_ERR_INVALID_ARG;
+  WsLayout L;
+  mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, out, B, Hq, Hkv, N, d, p_scale_mode, out_dtype,
+                                       workspace, workspace_bytes, &L);
+  if (s != MXATTN_OK) return s;
+  if (static_cast<uint64_t>(B) * Hq * N >= (1ull << 31)) return MXATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  const uint32_t tiles = static_cast<uint32_t>(L.npad / kTile);
+  const uint32_t nblk = static_cast<uint32_t>((N + 31) / 32);
+  const ScaleRepackParams reps[3] = {
+      {qs, w + L.qs, static_cast<uint32_t>(B * Hq), tiles, static_cast<uint32_t>(N), static_cast<uint32_t>(d / 32), 0},
+      {ks, w + L.ks, static_cast<uint32_t>(B * Hkv), tiles, static_cast<uint32_t>(N), static_cast<uint32_t>(d / 32), 0},
+      {vts, w + L.vs, static_cast<uint32_t>(B * Hkv), tiles, static_cast<uint32_t>(d), nblk, 1}};
+  for (const ScaleRepackParams& r : reps)
+    if (launch_repack_scales(r, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  const CodeSources src{qc, kc, vtc, N, static_cast<uint64_t>(nblk) * 16};
+  return attend_impl(out, B, Hq, Hkv, N, d, causal, p_scale_mode, pnq, out_dtype, workspace, st, L, src, -1, 0, 0,
+                     nullptr, nullptr);
 }
 
 mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
@@ -292,8 +337,8 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = prepare_impl(q, k, v, B, Hq, Hkv, N, d, scale_mode, workspace, workspace_bytes, st, L);
   if (s != MXATTN_OK) return s;
-  return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace, st, L, dbg_bh, dbg_r0,
-                     dbg_r1, p_codes, p_scales);
+  return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace, st, L,
+                     workspace_codes(workspace, L), dbg_bh, dbg_r0, dbg_r1, p_codes, p_scales);
 }
 
 mxattn_status mxattn_check_status(void* workspace, void* stream, unsigned int* detail) {

@@ -40,6 +40,18 @@ struct ColQuantParams {
 cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream);
 cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
 
+// Row-major scale bytes -> 512-byte MMA atoms [heads][tiles][512], zero where the source has no
+// element. transposed = 0: src [heads][rows][kb], atom t holds rows 128t.. and blocks 0..3;
+// transposed = 1 (V^T): src [heads][rows = channels][kb = key blocks], atom t holds channels
+// 0..127 and key blocks 4t..4t+3.
+struct ScaleRepackParams {
+  const uint8_t* src;
+  uint8_t* dst;
+  uint32_t heads, tiles, rows, kb;
+  int transposed;
+};
+cudaError_t launch_repack_scales(const ScaleRepackParams& p, cudaStream_t stream);
+
 struct AttnParams {
   const uint8_t* qsf;      // atom-tiled scales of Q  [B*Hq][Npad/128][512]
   const uint8_t* ksf;      // atom-tiled scales of K  [B*Hkv][Npad/128][512]
@@ -47,6 +59,7 @@ struct AttnParams {
   void* out;               // [B, Hq, N, d], fp32 or bf16
   int out_bf16;
   int B, Hq, Hkv, N, Npad, causal, mode, pnq;
+  int rows_per_head;       // row stride between heads in the Q / K code tensors (Npad or N)
   float scale_log2;        // log2(e) / sqrt(d)
   unsigned int* status;    // device status word (0 = ok)
   uint8_t* dbg_codes;      // optional P~ dump: [r1 - r0][Npad / 2]

@@ -100,6 +100,23 @@ def test_forward_argument_checks(lib):
     assert call(wsb=good - 1) == WORKSPACE
 
 
+def test_forward_quantized_argument_checks(lib):
+    f = lib.mxattn_forward_quantized
+    good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
+    ops = [FAKE] * 6
+
+    def call(ops=ops, out=FAKE, d=64, mode=1, wsb=good):
+        return f(*ops, out, 1, 2, 2, 256, d, 0, mode, 1, 0, FAKE, wsb, None)
+
+    assert call(ops=[None] + ops[1:]) == INVALID
+    assert call(out=None) == INVALID
+    assert call(ops=[FAKE + 8] + ops[1:]) == INVALID                  # codes must be 16-byte aligned
+    assert call(ops=ops[:4] + [FAKE + 4, FAKE]) == INVALID
+    assert call(ops=[FAKE, FAKE + 1] + ops[2:], wsb=good - 1) == WORKSPACE   # scales: any alignment
+    assert call(d=96) == UNSUPPORTED
+    assert call(mode=3) == INVALID
+
+
 def test_debug_argument_checks(lib):
     good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
     r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
