@@ -31,6 +31,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 FP4_PER_BF16 = 4.0          # nominal dense ratio: 9 PFLOP/s fp4 vs 2.25 PFLOP/s bf16
 ATTN_SOURCES = ["mxfp4_microscaled_bit_quantize_b200/csrc/attn_fwd_sm100.cu",
                 "mxfp4_microscaled_bit_quantize_b200/csrc/sm100_ptx.cuh"]
+GEMM_SOURCES = ["mxfp4_microscaled_bit_quantize_b200/csrc/gemm_sm100.cu",
+                "mxfp4_microscaled_bit_quantize_b200/csrc/sm100_ptx.cuh"]
 QUANT_SOURCES = ["mxfp4_microscaled_bit_quantize_b200/csrc/quantize.cu",
                  "mxfp4_microscaled_bit_quantize_b200/csrc/sm100_ptx.cuh"]
 
@@ -200,6 +202,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     if args.mode == "quantizer":
         run_quantizer_only(args, dev)
         return
+    if args.mode == "gemm":
+        run_gemm_only(args, dev)
+        return
     q, k, v = synthetic.attn_inputs(cfg)
     q_h, k_h, v_h = (t.pin_memory() for t in (q, k, v))
     dq, dk, dv = (t.to(dev) for t in (q_h, k_h, v_h))
@@ -282,6 +287,30 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     fq_ms = f_start.elapsed_time(f_stop) / fq_steps
     del fq_ops
 
+    # block-scaled MXFP4 GEMM (W4A4) on its own workload: A [M, K], B [N, K] quantized once
+    gm, gn, gk = synthetic.GEMM_SHAPE
+    ga = torch.randn((gm, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(5))
+    gb = torch.randn((gn, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(6))
+    g_ops = (*api.mxattn_quantize(ga.bfloat16(), False, api.SCALE_UOS),
+             *api.mxattn_quantize((gb * 0.05).bfloat16(), False, api.SCALE_UOS))
+    del ga, gb
+    g_ws = api.gemm_workspace(gm, gn, gk, dev)
+    g_out = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        api.mxattn_gemm(*g_ops, gk, out_dtype=torch.bfloat16, workspace=g_ws, out=g_out)
+    barrier()
+    g_start, g_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g_iters = 10
+    g_start.record(stream)
+    for _ in range(g_iters):
+        api.mxattn_gemm(*g_ops, gk, out_dtype=torch.bfloat16, workspace=g_ws, out=g_out)
+    g_stop.record(stream)
+    barrier()
+    if api.mxattn_check_status(g_ws) != 0:
+        raise RuntimeError("device pipeline timeout in the GEMM")
+    gemm_ms = g_start.elapsed_time(g_stop) / g_iters
+    del g_ops, g_ws, g_out
+
     # standalone quantizer on its own workload (65536 x 1024 bf16), two buffer sets > L2
     xq = [synthetic.quant_input().to(dev) for _ in range(2)]
     qbuf = [api.mxattn_quantize(x, False, api.SCALE_UOS) for x in xq]
@@ -299,8 +328,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
-    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms = reduce_max_over_ranks(
-        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms], world, dev)
+    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms = reduce_max_over_ranks(
+        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms], world, dev)
     if rank != 0:
         return
 
@@ -341,6 +370,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
         "forward_quantized": {"ms": fq_ms, "tflops": flops / (fq_ms * 1e-3) / 1e12,
                               "note": "mxattn_forward_quantized on pre-quantized Q/K/V: scale repack + kernel"},
+        "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
+                 "tflops": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12,
+                 "frac": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12 / fp4_peak,
+                 "traffic": profile_traffic("mxgemm_16384x16384x8192.json", sources_hash(GEMM_SOURCES))},
         "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 4 * args.steps,
@@ -353,6 +386,33 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                                 "sample": f"{args.cpu_rows} query rows of head 0 (that head's Q/K/V "
                                           f"quantized, attention over all {cfg.N} keys), {dt:.1f} s"}
     print(json.dumps(line), flush=True)
+
+
+def run_gemm_only(args, dev):
+    """The W4A4 GEMM alone (used for its Nsight Compute capture); --heads scales M down."""
+    import torch
+
+    from mxfp4_microscaled_bit_quantize_b200 import api, synthetic
+    gm, gn, gk = synthetic.GEMM_SHAPE
+    if args.heads:
+        gm = 128 * args.heads
+    ga = torch.randn((gm, gk), device=dev, generator=torch.Generator(dev).manual_seed(5)).bfloat16()
+    gb = (torch.randn((gn, gk), device=dev, generator=torch.Generator(dev).manual_seed(6)) * 0.05).bfloat16()
+    ops = (*api.mxattn_quantize(ga, False, api.SCALE_UOS), *api.mxattn_quantize(gb, False, api.SCALE_UOS))
+    ws = api.gemm_workspace(gm, gn, gk, dev)
+    out = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        api.mxattn_gemm(*ops, gk, out_dtype=torch.bfloat16, workspace=ws, out=out)
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        api.mxattn_gemm(*ops, gk, out_dtype=torch.bfloat16, workspace=ws, out=out)
+    e.record()
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / args.steps
+    print(json.dumps({"mode": "gemm", "M": gm, "N": gn, "K": gk, "ms": ms,
+                      "tflops": 2.0 * gm * gn * gk / (ms * 1e-3) / 1e12}), flush=True)
 
 
 def run_quantizer_only(args, dev):
@@ -385,7 +445,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["full", "attention", "quantizer"], default="full",
+    ap.add_argument("--mode", choices=["full", "attention", "quantizer", "gemm"], default="full",
                     help="attention / quantizer: time only that part (small cases for profiling)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
     args = ap.parse_args()

@@ -124,6 +124,25 @@ mxattn_status mxattn_forward_quantized(const uint8_t* qc, const uint8_t* qs, con
                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mxattn_gemm -- block-scaled MXFP4 matrix product C[M, N] = dq(A)[M, K] dq(B)[N, K]^T (both
+ * operands K-major, as W4A4 layers and the attention's Q K^T use them). The MX format is the
+ * "Quantization Error" page's (section "Where the error comes from"): E2M1 codes, one exact
+ * power-of-two scale per 32 elements; no counterpart of the attention's P~ step.
+ *   a_codes : [M, K/2] bytes, a_scales: [M, K/32] E8M0 bytes (mxattn_quantize of A, transpose = 0)
+ *   b_codes : [N, K/2] bytes, b_scales: [N, K/32]
+ *   c       : [M, N] fp32 (out_dtype = MXATTN_OUT_F32) or bf16, row-major, device
+ *   Codes and c 16-byte aligned; workspace 256-byte aligned, >= mxattn_gemm_workspace_size bytes
+ *   (it receives the scales in the tensor-core layout and the status word read by
+ *   mxattn_check_status). Supported: K % 32 == 0, N % 8 == 0, M, N, K < 2^31, M <= 65535 * 128.
+ *   Errors: null / misaligned pointers or bad dtype -> MXATTN_ERR_INVALID_ARG; other shapes ->
+ *   MXATTN_ERR_UNSUPPORTED; small workspace -> MXATTN_ERR_WORKSPACE. Asynchronous on stream.
+ */
+size_t mxattn_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                          const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The two halves of mxattn_forward, for callers that time or reuse them separately:
  *   mxattn_forward_prepare quantizes q, k, v into the workspace;
  *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same

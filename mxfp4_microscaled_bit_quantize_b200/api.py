@@ -139,6 +139,37 @@ def mxattn_forward_quantized(qc, qs, kc, ks, vtc, vts, N: int, d: int, causal: b
     return out
 
 
+def gemm_workspace(M: int, N: int, K: int, device) -> torch.Tensor:
+    n = int(_lib.load().mxattn_gemm_workspace_size(M, N, K))
+    if n == 0:
+        raise ValueError("unsupported GEMM shape (needs K % 32 == 0, N % 8 == 0)")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mxattn_gemm(a_codes, a_scales, b_codes, b_scales, K: int, out_dtype=torch.float32,
+                workspace: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] = dq(A) dq(B)^T for A, B in MXFP4 (codes [R, K/2], scales [R, K/32], uint8 CUDA)."""
+    for t, n in ((a_codes, "a_codes"), (a_scales, "a_scales"), (b_codes, "b_codes"), (b_scales, "b_scales")):
+        _need(t, n, torch.uint8)
+    M, N = int(a_codes.shape[0]), int(b_codes.shape[0])
+    for t, n, r, c in ((a_codes, "a_codes", M, K // 2), (a_scales, "a_scales", M, K // 32),
+                       (b_codes, "b_codes", N, K // 2), (b_scales, "b_scales", N, K // 32)):
+        if tuple(t.shape) != (r, c):
+            raise ValueError(f"{n} must have shape {(r, c)}, got {tuple(t.shape)}")
+    dt = torch.float32 if out_dtype in (OUT_F32, torch.float32) else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=a_codes.device)
+    else:
+        _need(out, "out", dt)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, a_codes.device)
+    st = _lib.load().mxattn_gemm(a_codes.data_ptr(), a_scales.data_ptr(), b_codes.data_ptr(), b_scales.data_ptr(),
+                                 out.data_ptr(), M, N, K, OUT_F32 if dt == torch.float32 else OUT_BF16,
+                                 workspace.data_ptr(), workspace.numel(), _stream(a_codes.device))
+    _lib.check(st, "mxattn_gemm")
+    return out
+
+
 def mxattn_forward_prepare(q, k, v, scale_mode: int, workspace: torch.Tensor) -> None:
     B, Hq, Hkv, N, d = _shapes(q, k, v)
     st = _lib.load().mxattn_forward_prepare(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d,

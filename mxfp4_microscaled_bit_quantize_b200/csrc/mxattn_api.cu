@@ -192,9 +192,80 @@ mxattn_status check_forward_args(const void* q, const void* k, const void* v, co
   return MXATTN_OK;
 }
 
+// GEMM workspace: status area, then the scale atoms of A and B [row tile][kgroup][512].
+struct GemmLayout {
+  size_t sfa, sfb, total;
+  int k_stages, kgroups, tiles_m, tiles_n128;
+};
+
+bool gemm_layout(int64_t M, int64_t N, int64_t K, GemmLayout* L) {
+  if (M < 1 || N < 1 || K < 32 || K % 32 != 0 || N % 8 != 0) return false;
+  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return false;
+  if ((M + 127) / 128 > 65535) return false;
+  L->k_stages = static_cast<int>((K + 255) / 256);
+  L->kgroups = 2 * L->k_stages;
+  L->tiles_m = static_cast<int>((M + 127) / 128);
+  L->tiles_n128 = 2 * static_cast<int>((N + 255) / 256);
+  size_t off = kAlign;
+  L->sfa = off;
+  off = align_up(off + static_cast<size_t>(L->tiles_m) * L->kgroups * 512, kAlign);
+  L->sfb = off;
+  off = align_up(off + static_cast<size_t>(L->tiles_n128) * L->kgroups * 512, kAlign);
+  L->total = off;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t mxattn_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  GemmLayout L;
+  return gemm_layout(M, N, K, &L) ? L.total : 0;
+}
+
+mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                          const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !c || !workspace) return MXATTN_ERR_INVALID_ARG;
+  if (out_dtype != MXATTN_OUT_F32 && out_dtype != MXATTN_OUT_BF16) return MXATTN_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1) return MXATTN_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(c, 16) || !aligned(workspace, 256))
+    return MXATTN_ERR_INVALID_ARG;
+  GemmLayout L;
+  if (!gemm_layout(M, N, K, &L)) return MXATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < L.total) return MXATTN_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  const uint32_t kb = static_cast<uint32_t>(K / 32);
+  const ScaleRepackParams reps[2] = {
+      {a_scales, w + L.sfa, 1u, static_cast<uint32_t>(L.tiles_m), static_cast<uint32_t>(M), kb, 0,
+       static_cast<uint32_t>(L.kgroups)},
+      {b_scales, w + L.sfb, 1u, static_cast<uint32_t>(L.tiles_n128), static_cast<uint32_t>(N), kb, 0,
+       static_cast<uint32_t>(L.kgroups)}};
+  for (const ScaleRepackParams& r : reps)
+    if (launch_repack_scales(r, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, a_codes, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M), 128, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tb, b_codes, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N), 128, 256,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return MXATTN_ERR_CUDA;
+  GemmParams p{};
+  p.sfa = w + L.sfa;
+  p.sfb = w + L.sfb;
+  p.c = c;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.k_stages = L.k_stages;
+  p.kgroups = L.kgroups;
+  p.out_bf16 = (out_dtype == MXATTN_OUT_BF16) ? 1 : 0;
+  p.status = reinterpret_cast<unsigned int*>(w);
+  return launch_gemm(ta, tb, p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
 
 int mxattn_version(void) { return 101; }
 

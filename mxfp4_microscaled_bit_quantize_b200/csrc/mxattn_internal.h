@@ -44,11 +44,14 @@ cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
 // element. transposed = 0: src [heads][rows][kb], atom t holds rows 128t.. and blocks 0..3;
 // transposed = 1 (V^T): src [heads][rows = channels][kb = key blocks], atom t holds channels
 // 0..127 and key blocks 4t..4t+3.
+// kgroups > 1 (transposed = 0 only): atoms [heads][tiles][kgroups][512], kgroup g holding blocks
+// 4g..4g+3 of the rows of its tile.
 struct ScaleRepackParams {
   const uint8_t* src;
   uint8_t* dst;
   uint32_t heads, tiles, rows, kb;
   int transposed;
+  uint32_t kgroups;
 };
 cudaError_t launch_repack_scales(const ScaleRepackParams& p, cudaStream_t stream);
 
@@ -69,6 +72,21 @@ struct AttnParams {
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const AttnParams& p, int d, cudaStream_t stream);
+
+// Block-scaled MXFP4 GEMM C[M, N] = dq(A) dq(B)^T; A, B codes are read through tensor maps, their
+// scales from atoms [row tile][kgroup][512] (kgroup = 128 K elements; B row tiles padded to even).
+struct GemmParams {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  void* c;                 // [M, N] fp32 or bf16, row-major
+  int M, N, K;
+  int k_stages;            // ceil(K / 256)
+  int kgroups;             // 2 * k_stages (atoms per row tile, zero-padded past K)
+  int out_bf16;
+  unsigned int* status;
+};
+
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, cudaStream_t stream);
 
 // Status codes written by kernels into the workspace status word.
 enum : unsigned int {

@@ -177,19 +177,22 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(ColQuantParams p) {
 
 // One thread per atom byte: invert atom_offset to find the (row, block) it holds.
 __global__ void __launch_bounds__(256) repack_scales_kernel(const ScaleRepackParams p) {
-  const uint64_t total = static_cast<uint64_t>(p.heads) * p.tiles * 512u;
+  const uint32_t kgroups = p.kgroups ? p.kgroups : 1u;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * p.tiles * kgroups * 512u;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     const uint32_t b = static_cast<uint32_t>(i & 511u);
     const uint64_t atom = i >> 9;
-    const uint32_t t = static_cast<uint32_t>(atom % p.tiles);
-    const uint64_t head = atom / p.tiles;
+    const uint32_t g = static_cast<uint32_t>(atom % kgroups);
+    const uint32_t t = static_cast<uint32_t>((atom / kgroups) % p.tiles);
+    const uint64_t head = atom / kgroups / p.tiles;
     const uint32_t r = ((b >> 4) & 31u) + 32u * ((b & 15u) >> 2);   // 0..127
     const uint32_t k = b & 3u;
     uint8_t v = 0;
     if (!p.transposed) {
       const uint32_t row = t * 128u + r;
-      if (row < p.rows && k < p.kb) v = p.src[(head * p.rows + row) * p.kb + k];
+      const uint32_t blk = g * 4u + k;
+      if (row < p.rows && blk < p.kb) v = p.src[(head * p.rows + row) * p.kb + blk];
     } else {
       const uint32_t blk = t * 4u + k;
       if (r < p.rows && blk < p.kb) v = p.src[(head * p.rows + r) * p.kb + blk];
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(256) repack_scales_kernel(const ScaleRepackPar
 }
 
 cudaError_t launch_repack_scales(const ScaleRepackParams& p, cudaStream_t stream) {
-  const uint64_t total = static_cast<uint64_t>(p.heads) * p.tiles * 512u;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * p.tiles * (p.kgroups ? p.kgroups : 1u) * 512u;
   if (total == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

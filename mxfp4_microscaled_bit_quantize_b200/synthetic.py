@@ -188,3 +188,44 @@ def quant_input(rows: int = QUANT_ROWS, cols: int = QUANT_COLS, seed: int = QUAN
     with ThreadPoolExecutor(max_workers=threads) as ex:
         list(ex.map(run, range(rows // chunk)))
     return out
+
+
+# ---------------------------------------------------------------- W4A4 GEMM operands
+# A (activations): N(0,1) rows with a per-row gain, log-uniform in [0.1, 10]; B (weights):
+# N(0, 0.05^2). In both, 0.1% of the entries are multiplied by 20 (outliers that set their
+# block's scale). Every row has its own stream, so the oracle regenerates only sampled rows.
+GEMM_SHAPE = (16384, 16384, 8192)       # M, N, K of the benchmark's product
+GEMM_SEED = 5
+_GEMM_TAG = {"A": 21, "B": 22}
+
+
+def gemm_rows_f32(which: str, rows, K: int, seed: int = GEMM_SEED) -> np.ndarray:
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    out = np.empty((rows.size, K), dtype=np.float32)
+    for i, r in enumerate(rows):
+        rng = _rng(seed, _GEMM_TAG[which], int(r))
+        x = rng.standard_normal(K, dtype=np.float32)
+        if which == "A":
+            x *= np.float32(10.0 ** rng.uniform(-1.0, 1.0))
+        else:
+            x *= np.float32(0.05)
+        x[rng.random(K) < 0.001] *= 20.0
+        out[i] = x
+    return out
+
+
+def gemm_inputs(M: int, N: int, K: int, seed: int = GEMM_SEED, threads: int = 8):
+    """(A bf16 [M, K], B bf16 [N, K]) as contiguous CPU tensors."""
+    a = torch.empty((M, K), dtype=torch.bfloat16)
+    b = torch.empty((N, K), dtype=torch.bfloat16)
+    step = 1024
+
+    def run(job):
+        which, r0, dst, rows = job
+        r1 = min(r0 + step, rows)
+        dst[r0:r1].copy_(_to_bf16(gemm_rows_f32(which, np.arange(r0, r1), K, seed)))
+
+    jobs = [("A", r0, a, M) for r0 in range(0, M, step)] + [("B", r0, b, N) for r0 in range(0, N, step)]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(run, jobs))
+    return a, b

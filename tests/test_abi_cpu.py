@@ -117,6 +117,38 @@ def test_forward_quantized_argument_checks(lib):
     assert call(mode=3) == INVALID
 
 
+def _gemm_ws_mirror(M, N, K):
+    up = lambda x, a: -(-x // a) * a  # noqa: E731
+    kst = -(-K // 256)
+    off = 1024
+    for rows in (-(-M // 128), 2 * -(-N // 256)):
+        off = up(off + rows * 2 * kst * 512, 1024)
+    return off
+
+
+def test_gemm_workspace_and_argument_checks(lib):
+    ws = lib.mxattn_gemm_workspace_size
+    for shape in [(1, 8, 32), (300, 520, 992), (16384, 16384, 8192)]:
+        assert ws(*shape) == _gemm_ws_mirror(*shape)
+    assert ws(4, 8, 48) == 0          # K % 32 != 0
+    assert ws(4, 12, 64) == 0         # N % 8 != 0
+    g = lib.mxattn_gemm
+    good = ws(256, 256, 512)
+    ok = dict(a=FAKE, sa=FAKE, b=FAKE, sb=FAKE, c=FAKE, M=256, N=256, K=512, od=0, w=FAKE, wb=good)
+
+    def call(**kw):
+        x = dict(ok, **kw)
+        return g(x["a"], x["sa"], x["b"], x["sb"], x["c"], x["M"], x["N"], x["K"], x["od"], x["w"], x["wb"], None)
+
+    assert call(a=None) == INVALID
+    assert call(b=FAKE + 8) == INVALID
+    assert call(c=FAKE + 4) == INVALID
+    assert call(od=3) == INVALID
+    assert call(K=100) == UNSUPPORTED
+    assert call(N=250) == UNSUPPORTED
+    assert call(wb=good - 1) == WORKSPACE
+
+
 def test_debug_argument_checks(lib):
     good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
     r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
