@@ -78,6 +78,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+// 2-D tensor map of the given element type over a row-major matrix (dims and box in elements).
+bool make_map_typed(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, uint64_t cols, uint64_t rows,
+                    uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                            int scale_mode, void* ws, size_t ws_bytes, cudaStream_t st, const WsLayout& L) {
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -246,12 +260,20 @@ mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
        static_cast<uint32_t>(L.kgroups)}};
   for (const ScaleRepackParams& r : reps)
     if (launch_repack_scales(r, st) != cudaSuccess) return MXATTN_ERR_CUDA;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_map(&ta, a_codes, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M), 128, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tb, b_codes, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N), 128, 256,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return MXATTN_ERR_CUDA;
+  if (out_dtype == MXATTN_OUT_BF16) {
+    // C as [M, N] bf16 for the epilogue's TMA stores: 128 rows x 64 columns per box, 128B swizzle
+    if (!make_map_typed(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                        static_cast<uint64_t>(N) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MXATTN_ERR_CUDA;
+  } else {
+    std::memset(&tc, 0, sizeof(tc));   // fp32 output is stored without TMA
+  }
   GemmParams p{};
   p.sfa = w + L.sfa;
   p.sfb = w + L.sfb;
@@ -263,7 +285,7 @@ mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
   p.kgroups = L.kgroups;
   p.out_bf16 = (out_dtype == MXATTN_OUT_BF16) ? 1 : 0;
   p.status = reinterpret_cast<unsigned int*>(w);
-  return launch_gemm(ta, tb, p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+  return launch_gemm(ta, tb, tc, p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
 

@@ -86,7 +86,8 @@ struct GemmParams {
   unsigned int* status;
 };
 
-cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, cudaStream_t stream);
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, const GemmParams& p,
+                        cudaStream_t stream);
 
 // Status codes written by kernels into the workspace status word.
 enum : unsigned int {
