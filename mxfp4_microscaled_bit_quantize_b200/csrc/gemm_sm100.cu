@@ -18,10 +18,10 @@
 //              stage, i.e. after its MMAs completed), then 4 x tcgen05.mma kind::mxf4.block_scale
 //              (M = 128, N = 256, K = 64) per stage. A tile starts once the epilogue has drained
 //              the previous tile's accumulator.
-//   warps 2-5  epilogue, one accumulator row per thread. bf16: tcgen05.ld, convert and write a
-//              128-byte-swizzled staging tile in shared memory, release the accumulator, then one
-//              thread stores the tile with TMA while the next tile's MMAs run. fp32: direct row
-//              stores, then release.
+//   warps 2-5  epilogue, one accumulator row per thread. bf16: tcgen05.ld the whole row into
+//              registers (packed bf16), release the accumulator, then stream the row out through a
+//              128-byte-swizzled staging box in shared memory, one TMA store per 64 columns, while
+//              the next tile's MMAs run. fp32: direct row stores, then release.
 // TMEM: accumulator columns [0, 256), scale columns from 256 (kGStages x 24).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -37,7 +37,7 @@ constexpr int kGm = 128;              // rows of A per tile
 constexpr int kGn = 256;              // rows of B (columns of C) per tile
 constexpr int kGk = 256;              // K elements per stage
 constexpr int kGkBytes = kGk / 2;     // 128 bytes of codes per row per stage
-constexpr int kGStages = 3;
+constexpr int kGStages = 4;
 constexpr int kGroupM = 8;            // tile rows per raster group
 constexpr int kGThreads = 192;
 constexpr uint32_t kGTmemCols = 512;
@@ -49,15 +49,15 @@ constexpr int kCBoxCols = 64;         // bf16 columns per TMA store box (128 byt
 struct __align__(1024) GemmSmem {
   uint8_t a[kGStages][kGm * kGkBytes];     // 16 KiB per stage
   uint8_t b[kGStages][kGn * kGkBytes];     // 32 KiB per stage
-  uint8_t c[kGn / kCBoxCols][kGm * 128];   // bf16 staging tile: 4 boxes of 128 rows x 64 columns
+  uint8_t c[kGm * 128];                    // bf16 staging box: 128 rows x 64 columns, 128B swizzle
   uint8_t sfa[kGStages][2][512];           // [kgroup] atom of the 128 A rows
   uint8_t sfb[kGStages][2][2][512];        // [row tile][kgroup]
   uint64_t full[kGStages];
   uint64_t empty[kGStages];
   uint64_t acc_full;                       // MMA -> epilogue, once per tile
   uint64_t acc_empty;                      // epilogue (128 threads) -> MMA, once per tile
-  uint64_t c_written;                      // epilogue threads (128) -> store thread
-  uint64_t c_free;                         // store thread -> epilogue: staging tile read by TMA
+  uint64_t c_written;                      // epilogue threads (128) -> store thread, once per box
+  uint64_t c_free;                         // store thread -> epilogue: staging box read by TMA
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -163,6 +163,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
     auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
     constexpr uint32_t idesc0 = idesc_mxf4(kGn, 0, 0);
     constexpr uint32_t idesc1 = idesc_mxf4(kGn, 2, 2);
+    // per-stage descriptors, computed once: a K step inside the 128-byte swizzled rows only adds
+    // (offset >> 4) to the start-address field (shared addresses stay below 2^18, no carry)
+    uint64_t desc_a[kGStages], desc_b[kGStages], desc_sfa[kGStages][2], desc_sfb[kGStages][2][2];
+#pragma unroll
+    for (int st = 0; st < kGStages; ++st) {
+      desc_a[st] = smem_desc(smem_u32(s.a[st]), 0, 8 * kGkBytes, kLayoutSw128);
+      desc_b[st] = smem_desc(smem_u32(s.b[st]), 0, 8 * kGkBytes, kLayoutSw128);
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        desc_sfa[st][g] = sf_desc(s.sfa[st][g]);
+        desc_sfb[st][0][g] = sf_desc(s.sfb[st][0][g]);
+        desc_sfb[st][1][g] = sf_desc(s.sfb[st][1][g]);
+      }
+    }
     bool ok = true;
     int it = 0, i = 0;
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++i) {
@@ -179,19 +193,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (leader) {
-          const uint32_t a0 = smem_u32(s.a[st]), b0 = smem_u32(s.b[st]);
+          uint64_t da = 0, db = 0, dsa[2] = {0, 0}, dsb[2][2] = {{0, 0}, {0, 0}};
+#pragma unroll
+          for (int q = 0; q < kGStages; ++q) {   // select this stage's descriptors without local memory
+            if (q == st) {
+              da = desc_a[q];
+              db = desc_b[q];
+              dsa[0] = desc_sfa[q][0];
+              dsa[1] = desc_sfa[q][1];
+              dsb[0][0] = desc_sfb[q][0][0];
+              dsb[0][1] = desc_sfb[q][0][1];
+              dsb[1][0] = desc_sfb[q][1][0];
+              dsb[1][1] = desc_sfb[q][1][1];
+            }
+          }
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
             const uint32_t sfa = tmem + kGColSf + st * 24 + g * 12, sfb = sfa + 4;
-            tc_cp_sf(sfa, sf_desc(s.sfa[st][g]));
-            tc_cp_sf(sfb, sf_desc(s.sfb[st][0][g]));
-            tc_cp_sf(sfb + 4, sf_desc(s.sfb[st][1][g]));
+            tc_cp_sf(sfa, dsa[g]);
+            tc_cp_sf(sfb, dsb[0][g]);
+            tc_cp_sf(sfb + 4, dsb[1][g]);
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
-              const uint32_t off = g * 64 + kk * 32;
-              const uint64_t ad = smem_desc(a0 + off, 0, 8 * kGkBytes, kLayoutSw128);
-              const uint64_t bd = smem_desc(b0 + off, 0, 8 * kGkBytes, kLayoutSw128);
-              tc_mma_mxf4(tmem + kGColAcc, ad, bd, kk ? idesc1 : idesc0, sfa, sfb, (kt | g | kk) != 0 ? 1u : 0u);
+              const uint64_t off = static_cast<uint64_t>((g * 64 + kk * 32) >> 4);
+              tc_mma_mxf4(tmem + kGColAcc, da + off, db + off, kk ? idesc1 : idesc0, sfa, sfb,
+                          (kt | g | kk) != 0 ? 1u : 0u);
             }
           }
           tc_commit(&s.empty[st]);   // the stage's smem and scale columns are free once these MMAs end
@@ -223,47 +249,48 @@ __global__ void __launch_bounds__(kGThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.acc_full, i & 1, abort_flag, p.status, kStatusTimeoutPV | 1));
       if (!ok) break;
       if (p.out_bf16) {
-        if (i > 0) {   // the previous tile's stores must have read the staging tile
-          ok = __all_sync(0xffffffffu, mbar_wait(&s.c_free, (i - 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 2));
-          if (!ok) break;
-        }
         tc_fence_after();
-#pragma unroll 1
+        uint32_t packed[kGn / 2];            // the row as bf16 pairs
+#pragma unroll
         for (int cc = 0; cc < kGn / 32; ++cc) {
           uint32_t raw[32];
           tmem_ld32(tmem + lane_addr + kGColAcc + cc * 32, raw);
           tc_wait_ld();
-          uint8_t* box = s.c[cc >> 1] + r * 128;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[q * 8 + 2 * u]),
-                                                              __uint_as_float(raw[q * 8 + 2 * u + 1]));
-              w[u] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            const uint32_t j = static_cast<uint32_t>((cc & 1) * 4 + q);
-            *reinterpret_cast<uint4*>(box + ((j ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int u = 0; u < 16; ++u) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[2 * u]), __uint_as_float(raw[2 * u + 1]));
+            packed[cc * 16 + u] = *reinterpret_cast<const uint32_t*>(&h2);
           }
         }
         tc_fence_before();
         mbar_arrive(&s.acc_empty);           // the MMAs of the next tile may overwrite TMEM now
-        fence_proxy_async_smem();            // staging writes -> visible to the TMA store
-        mbar_arrive(&s.c_written);
-        if (store_thread) {
-          if (mbar_wait(&s.c_written, i & 1, abort_flag, p.status, kStatusTimeoutPV | 3)) {
+        uint8_t* row_base = s.c + r * 128;
 #pragma unroll
-            for (int b = 0; b < kGn / kCBoxCols; ++b) {
-              const int x = tn * kGn + b * kCBoxCols;
-              if (x < p.N) tma_store_2d(&tmC, s.c[b], x, tm * kGm);
-            }
-            bulk_commit_group();
-            bulk_wait_group_read0();
-            mbar_arrive(&s.c_free);
+        for (int b = 0; b < kGn / kCBoxCols; ++b) {
+          const int seq = i * (kGn / kCBoxCols) + b;   // staging box uses so far
+          if (seq > 0) {   // the previous store must have read the staging box
+            ok = __all_sync(0xffffffffu, mbar_wait(&s.c_free, (seq - 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 2));
+            if (!ok) break;
           }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* w = packed + b * 32 + j * 4;
+            *reinterpret_cast<uint4*>(row_base + ((static_cast<uint32_t>(j) ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();          // staging writes -> visible to the TMA store
+          mbar_arrive(&s.c_written);
+          if (store_thread) {
+            if (mbar_wait(&s.c_written, seq & 1, abort_flag, p.status, kStatusTimeoutPV | 3)) {
+              const int x = tn * kGn + b * kCBoxCols;
+              if (x < p.N) tma_store_2d(&tmC, s.c, x, tm * kGm);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+              mbar_arrive(&s.c_free);
+            }
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        if (!ok) break;
       } else {
         tc_fence_after();
         const int row = tm * kGm + r;
