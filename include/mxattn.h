@@ -143,6 +143,18 @@ mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mxattn_selftest_wait_timeout -- exercises the failure detection every pipeline kernel uses; no
+ * counterpart in the pages. Launches one CTA whose mbarrier phase never completes: its first warp
+ * gives up after the library's wait bound (2 s of device time), writes 0x701 into the status word
+ * and raises the CTA's abort flag; its second warp, waiting on the same phase, leaves through the
+ * flag. Word 1 of the workspace then holds 3 (bit 0: the bounded wait returned, bit 1: the flag
+ * was seen). workspace: >= 256 bytes of device memory, 256-byte aligned; its first 256 bytes are
+ * overwritten. mxattn_check_status afterwards returns MXATTN_ERR_TIMEOUT with detail 0x701.
+ * The kernel neither faults nor traps, and the context stays usable.
+ */
+mxattn_status mxattn_selftest_wait_timeout(void* workspace, void* stream);
+
+/*
  * The two halves of mxattn_forward, for callers that time or reuse them separately:
  *   mxattn_forward_prepare quantizes q, k, v into the workspace;
  *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same

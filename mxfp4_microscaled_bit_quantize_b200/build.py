@@ -10,7 +10,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libmxattn.so")
-SOURCES = ["quantize.cu", "attn_fwd_sm100.cu", "gemm_sm100.cu", "mxattn_api.cu", "mxattn_noalloc.cu"]
+SOURCES = ["quantize.cu", "attn_fwd_sm100.cu", "gemm_sm100.cu", "mxattn_api.cu", "mxattn_noalloc.cu", "selftest.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -434,6 +434,14 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
                      workspace_codes(workspace, L), dbg_bh, dbg_r0, dbg_r1, p_codes, p_scales);
 }
 
+mxattn_status mxattn_selftest_wait_timeout(void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return MXATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* w = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  return launch_wait_timeout_selftest(w, w + 1, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
 mxattn_status mxattn_check_status(void* workspace, void* stream, unsigned int* detail) {
   if (!workspace) return MXATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

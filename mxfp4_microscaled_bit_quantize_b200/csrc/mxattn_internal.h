@@ -97,6 +97,9 @@ enum : unsigned int {
   kStatusTimeoutP = 0x400,
   kStatusTimeoutPV = 0x500,
   kStatusTimeoutEmpty = 0x600,
+  kStatusSelfTest = 0x700,
 };
+
+cudaError_t launch_wait_timeout_selftest(unsigned int* status, unsigned int* seen, cudaStream_t stream);
 
 }  // namespace mxattn
