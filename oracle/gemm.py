@@ -22,6 +22,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import mxfp4 as mx
+from . import nvfp4 as nv
 
 
 def mxgemm(a_codes, a_scales, b_codes, b_scales, K: int) -> np.ndarray:
@@ -36,3 +37,12 @@ def mxgemm_abs(a_codes, a_scales, b_codes, b_scales, K: int) -> np.ndarray:
     ad = np.abs(mx.dequantize_rows(a_codes, a_scales, K))
     bd = np.abs(mx.dequantize_rows(b_codes, b_scales, K))
     return ad @ bd.T
+
+
+def nvgemm(a_codes, a_scales, b_codes, b_scales, K: int) -> np.ndarray:
+    """C = dq(A) dq(B)^T in fp64 for A [M, K] and B [N, K] in NVFP4 (blocks of 16, E4M3 scales)."""
+    return nv.dequantize_rows(a_codes, a_scales, K) @ nv.dequantize_rows(b_codes, b_scales, K).T
+
+
+def nvgemm_abs(a_codes, a_scales, b_codes, b_scales, K: int) -> np.ndarray:
+    return np.abs(nv.dequantize_rows(a_codes, a_scales, K)) @ np.abs(nv.dequantize_rows(b_codes, b_scales, K)).T
