@@ -155,6 +155,26 @@ mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
 mxattn_status mxattn_selftest_wait_timeout(void* workspace, void* stream);
 
 /*
+ * NVFP4 comparison path (MXAttention abstract: MXFP4 attention is compared with NVFP4-based
+ * baselines; the pages give no NVFP4 recipe). Reading taken: blocks of 16 E2M1 elements along the
+ * contiguous axis, one unsigned FP8 E4M3 scale per block, s = E4M3(amax / 6) rounded to nearest-
+ * even and saturated at 448, elements x / s rounded to nearest-even on the E2M1 grid (saturating
+ * at 6), no tensor-level scale; both quotients are correctly rounded fp32 divisions.
+ *
+ * mxattn_quantize_nvfp4: x bf16 device [rows, cols] -> codes [rows, ceil(cols/16)*8] bytes
+ *   (element 2i in the low nibble; 8-byte aligned), scales [rows, ceil(cols/16)] E4M3 bytes.
+ *   Empty inputs are a no-op; null or misaligned pointers -> MXATTN_ERR_INVALID_ARG.
+ * mxattn_gemm_nvfp4: as mxattn_gemm with NVFP4 operands (scales [M, K/16] and [N, K/16]);
+ *   workspace from mxattn_gemm_nvfp4_workspace_size; same shape rules and errors.
+ */
+mxattn_status mxattn_quantize_nvfp4(const void* x, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
+                                    void* stream);
+size_t mxattn_gemm_nvfp4_workspace_size(int64_t M, int64_t N, int64_t K);
+mxattn_status mxattn_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                                const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The two halves of mxattn_forward, for callers that time or reuse them separately:
  *   mxattn_forward_prepare quantizes q, k, v into the workspace;
  *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same

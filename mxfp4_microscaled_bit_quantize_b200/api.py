@@ -170,6 +170,50 @@ def mxattn_gemm(a_codes, a_scales, b_codes, b_scales, K: int, out_dtype=torch.fl
     return out
 
 
+def mxattn_quantize_nvfp4(x: torch.Tensor):
+    """NVFP4-quantize a bf16 CUDA matrix [rows, cols] (blocks of 16, E4M3 scales):
+    codes [rows, ceil(cols/16)*8], scales [rows, ceil(cols/16)]."""
+    _need(x, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be [rows, cols]")
+    rows, cols = int(x.shape[0]), int(x.shape[1])
+    nb = -(-cols // 16)
+    codes = torch.empty((rows, nb * 8), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, nb), dtype=torch.uint8, device=x.device)
+    st = _lib.load().mxattn_quantize_nvfp4(x.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                                           _stream(x.device))
+    _lib.check(st, "mxattn_quantize_nvfp4")
+    return codes, scales
+
+
+def mxattn_gemm_nvfp4(a_codes, a_scales, b_codes, b_scales, K: int, out_dtype=torch.float32,
+                      workspace: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] = dq(A) dq(B)^T for A, B in NVFP4 (codes [R, K/2], E4M3 scales [R, K/16])."""
+    for t, n in ((a_codes, "a_codes"), (a_scales, "a_scales"), (b_codes, "b_codes"), (b_scales, "b_scales")):
+        _need(t, n, torch.uint8)
+    M, N = int(a_codes.shape[0]), int(b_codes.shape[0])
+    for t, n, r, c in ((a_codes, "a_codes", M, K // 2), (a_scales, "a_scales", M, K // 16),
+                       (b_codes, "b_codes", N, K // 2), (b_scales, "b_scales", N, K // 16)):
+        if tuple(t.shape) != (r, c):
+            raise ValueError(f"{n} must have shape {(r, c)}, got {tuple(t.shape)}")
+    dt = torch.float32 if out_dtype in (OUT_F32, torch.float32) else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=a_codes.device)
+    else:
+        _need(out, "out", dt)
+    lib = _lib.load()
+    if workspace is None:
+        n = int(lib.mxattn_gemm_nvfp4_workspace_size(M, N, K))
+        if n == 0:
+            raise ValueError("unsupported GEMM shape (needs K % 32 == 0, N % 8 == 0)")
+        workspace = torch.empty(n, dtype=torch.uint8, device=a_codes.device)
+    st = lib.mxattn_gemm_nvfp4(a_codes.data_ptr(), a_scales.data_ptr(), b_codes.data_ptr(), b_scales.data_ptr(),
+                               out.data_ptr(), M, N, K, OUT_F32 if dt == torch.float32 else OUT_BF16,
+                               workspace.data_ptr(), workspace.numel(), _stream(a_codes.device))
+    _lib.check(st, "mxattn_gemm_nvfp4")
+    return out
+
+
 def mxattn_forward_prepare(q, k, v, scale_mode: int, workspace: torch.Tensor) -> None:
     B, Hq, Hkv, N, d = _shapes(q, k, v)
     st = _lib.load().mxattn_forward_prepare(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d,

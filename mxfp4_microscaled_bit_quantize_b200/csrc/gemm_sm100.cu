@@ -37,23 +37,34 @@ constexpr int kGm = 128;              // rows of A per tile
 constexpr int kGn = 256;              // rows of B (columns of C) per tile
 constexpr int kGk = 256;              // K elements per stage
 constexpr int kGkBytes = kGk / 2;     // 128 bytes of codes per row per stage
-constexpr int kGStages = 4;
 constexpr int kGroupM = 8;            // tile rows per raster group
 constexpr int kGThreads = 192;
 constexpr uint32_t kGTmemCols = 512;
 constexpr uint32_t kGColAcc = 0;
-constexpr uint32_t kGColSf = 256;     // + stage * 24 + kgroup * 12: SFA 4 columns, SFB 8 columns
+constexpr uint32_t kGColSf = 256;     // + stage * kKg * 12 + kgroup * 12: SFA 4 columns, SFB 8 columns
 constexpr uint32_t kLayoutSw128 = 2;  // shared-memory descriptor layout code of the 128-byte swizzle
 constexpr int kCBoxCols = 64;         // bf16 columns per TMA store box (128 bytes)
 
+// Per format: MXFP4 (blocks of 32, UE8M0): a scale atom covers 128 K elements, two per stage, two
+// K = 64 MMAs per atom. NVFP4 (blocks of 16, UE4M3): an atom covers 64 K elements, four per stage,
+// one MMA per atom; its larger scale footprint leaves room for one stage less.
+template <bool NV>
+struct GemmFmt {
+  static constexpr int kStages = NV ? 3 : 4;
+  static constexpr int kKg = NV ? 4 : 2;          // scale atoms (K groups) per stage
+  static constexpr int kMmaPerKg = NV ? 1 : 2;
+};
+
+template <bool NV>
 struct __align__(1024) GemmSmem {
-  uint8_t a[kGStages][kGm * kGkBytes];     // 16 KiB per stage
-  uint8_t b[kGStages][kGn * kGkBytes];     // 32 KiB per stage
+  static constexpr int S = GemmFmt<NV>::kStages, G = GemmFmt<NV>::kKg;
+  uint8_t a[S][kGm * kGkBytes];            // 16 KiB per stage
+  uint8_t b[S][kGn * kGkBytes];            // 32 KiB per stage
   uint8_t c[kGm * 128];                    // bf16 staging box: 128 rows x 64 columns, 128B swizzle
-  uint8_t sfa[kGStages][2][512];           // [kgroup] atom of the 128 A rows
-  uint8_t sfb[kGStages][2][2][512];        // [row tile][kgroup]
-  uint64_t full[kGStages];
-  uint64_t empty[kGStages];
+  uint8_t sfa[S][G][512];                  // [kgroup] atom of the 128 A rows
+  uint8_t sfb[S][2][G][512];               // [row tile][kgroup]
+  uint64_t full[S];
+  uint64_t empty[S];
   uint64_t acc_full;                       // MMA -> epilogue, once per tile
   uint64_t acc_empty;                      // epilogue (128 threads) -> MMA, once per tile
   uint64_t c_written;                      // epilogue threads (128) -> store thread, once per box
@@ -62,8 +73,9 @@ struct __align__(1024) GemmSmem {
   int abort_flag;
 };
 
-constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
-static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
+template <bool NV>
+constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<NV>) + 1024; }
+static_assert(gemm_smem_bytes<false>() <= 232448 && gemm_smem_bytes<true>() <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ void gemm_drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
@@ -83,11 +95,16 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   tn = r / gm;
 }
 
+template <bool NV>
 __global__ void __launch_bounds__(kGThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  constexpr int kGStages = GemmFmt<NV>::kStages;
+  constexpr int kKg = GemmFmt<NV>::kKg;
+  constexpr uint32_t kSfBytes = 3u * kKg * 512u;   // A atoms + two row tiles of B atoms per stage
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem& s = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmSmem<NV>& s =
+      *reinterpret_cast<GemmSmem<NV>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_k = p.k_stages;
@@ -137,14 +154,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
           if (!ok) break;
         }
         if (leader) {
-          mbar_arrive_expect_tx(&s.full[st], kGm * kGkBytes + kGn * kGkBytes + 3 * 1024);
+          mbar_arrive_expect_tx(&s.full[st], kGm * kGkBytes + kGn * kGkBytes + kSfBytes);
           tma_load_2d(s.a[st], &tmA, &s.full[st], kt * kGkBytes, tm * kGm);
           tma_load_2d(s.b[st], &tmB, &s.full[st], kt * kGkBytes, tn * kGn);
-          // atoms [row tile][kgroup][512]: the two kgroups of this stage are adjacent
-          const size_t kg = static_cast<size_t>(2 * kt);
-          bulk_load(s.sfa[st][0], p.sfa + (static_cast<size_t>(tm) * p.kgroups + kg) * 512, 1024, &s.full[st]);
+          // atoms [row tile][kgroup][512]: the kgroups of this stage are adjacent
+          const size_t kg = static_cast<size_t>(kKg) * kt;
+          bulk_load(s.sfa[st][0], p.sfa + (static_cast<size_t>(tm) * p.kgroups + kg) * 512, kKg * 512, &s.full[st]);
           for (int rt = 0; rt < 2; ++rt)
-            bulk_load(s.sfb[st][rt][0], p.sfb + (static_cast<size_t>(2 * tn + rt) * p.kgroups + kg) * 512, 1024,
+            bulk_load(s.sfb[st][rt][0], p.sfb + (static_cast<size_t>(2 * tn + rt) * p.kgroups + kg) * 512, kKg * 512,
                       &s.full[st]);
         }
         __syncwarp();
@@ -161,17 +178,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const bool leader = elect_one_sync();
     const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
     auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
-    constexpr uint32_t idesc0 = idesc_mxf4(kGn, 0, 0);
+    constexpr uint32_t idesc0 = NV ? idesc_nvf4(kGn) : idesc_mxf4(kGn, 0, 0);
     constexpr uint32_t idesc1 = idesc_mxf4(kGn, 2, 2);
     // per-stage descriptors, computed once: a K step inside the 128-byte swizzled rows only adds
     // (offset >> 4) to the start-address field (shared addresses stay below 2^18, no carry)
-    uint64_t desc_a[kGStages], desc_b[kGStages], desc_sfa[kGStages][2], desc_sfb[kGStages][2][2];
+    uint64_t desc_a[kGStages], desc_b[kGStages], desc_sfa[kGStages][kKg], desc_sfb[kGStages][2][kKg];
 #pragma unroll
     for (int st = 0; st < kGStages; ++st) {
       desc_a[st] = smem_desc(smem_u32(s.a[st]), 0, 8 * kGkBytes, kLayoutSw128);
       desc_b[st] = smem_desc(smem_u32(s.b[st]), 0, 8 * kGkBytes, kLayoutSw128);
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
+      for (int g = 0; g < kKg; ++g) {
         desc_sfa[st][g] = sf_desc(s.sfa[st][g]);
         desc_sfb[st][0][g] = sf_desc(s.sfb[st][0][g]);
         desc_sfb[st][1][g] = sf_desc(s.sfb[st][1][g]);
@@ -193,31 +210,37 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (leader) {
-          uint64_t da = 0, db = 0, dsa[2] = {0, 0}, dsb[2][2] = {{0, 0}, {0, 0}};
+          uint64_t da = 0, db = 0, dsa[kKg], dsb[2][kKg];
+#pragma unroll
+          for (int g = 0; g < kKg; ++g) dsa[g] = dsb[0][g] = dsb[1][g] = 0;
 #pragma unroll
           for (int q = 0; q < kGStages; ++q) {   // select this stage's descriptors without local memory
             if (q == st) {
               da = desc_a[q];
               db = desc_b[q];
-              dsa[0] = desc_sfa[q][0];
-              dsa[1] = desc_sfa[q][1];
-              dsb[0][0] = desc_sfb[q][0][0];
-              dsb[0][1] = desc_sfb[q][0][1];
-              dsb[1][0] = desc_sfb[q][1][0];
-              dsb[1][1] = desc_sfb[q][1][1];
+#pragma unroll
+              for (int g = 0; g < kKg; ++g) {
+                dsa[g] = desc_sfa[q][g];
+                dsb[0][g] = desc_sfb[q][0][g];
+                dsb[1][g] = desc_sfb[q][1][g];
+              }
             }
           }
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint32_t sfa = tmem + kGColSf + st * 24 + g * 12, sfb = sfa + 4;
+          for (int g = 0; g < kKg; ++g) {
+            const uint32_t sfa = tmem + kGColSf + (st * kKg + g) * 12, sfb = sfa + 4;
             tc_cp_sf(sfa, dsa[g]);
             tc_cp_sf(sfb, dsb[0][g]);
             tc_cp_sf(sfb + 4, dsb[1][g]);
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint64_t off = static_cast<uint64_t>((g * 64 + kk * 32) >> 4);
-              tc_mma_mxf4(tmem + kGColAcc, da + off, db + off, kk ? idesc1 : idesc0, sfa, sfb,
-                          (kt | g | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < GemmFmt<NV>::kMmaPerKg; ++kk) {
+              // K offset of this instruction inside the 128-byte rows: 64 K elements = 32 bytes
+              const uint64_t off = static_cast<uint64_t>((g * 32 * GemmFmt<NV>::kMmaPerKg + kk * 32) >> 4);
+              if constexpr (NV)
+                tc_mma_nvf4(tmem + kGColAcc, da + off, db + off, idesc0, sfa, sfb, (kt | g) != 0 ? 1u : 0u);
+              else
+                tc_mma_mxf4(tmem + kGColAcc, da + off, db + off, kk ? idesc1 : idesc0, sfa, sfb,
+                            (kt | g | kk) != 0 ? 1u : 0u);
             }
           }
           tc_commit(&s.empty[st]);   // the stage's smem and scale columns are free once these MMAs end
@@ -331,20 +354,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, const GemmParams& p,
-                        cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kGemmSmemBytes));
+template <bool NV>
+cudaError_t launch_gemm_fmt(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                            const GemmParams& p, cudaStream_t stream) {
+  constexpr size_t smem = gemm_smem_bytes<NV>();
+  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long tiles = static_cast<long>((p.M + kGm - 1) / kGm) * ((p.N + kGn - 1) / kGn);
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  mxgemm_kernel<<<grid, kGThreads, kGemmSmemBytes, stream>>>(tmA, tmB, tmC, p);
+  mxgemm_kernel<NV><<<grid, kGThreads, smem, stream>>>(tmA, tmB, tmC, p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC, const GemmParams& p,
+                        cudaStream_t stream) {
+  return p.nvfp4 ? launch_gemm_fmt<true>(tmA, tmB, tmC, p, stream) : launch_gemm_fmt<false>(tmA, tmB, tmC, p, stream);
 }
 
 }  // namespace mxattn

@@ -212,12 +212,12 @@ struct GemmLayout {
   int k_stages, kgroups, tiles_m, tiles_n128;
 };
 
-bool gemm_layout(int64_t M, int64_t N, int64_t K, GemmLayout* L) {
+bool gemm_layout(int64_t M, int64_t N, int64_t K, GemmLayout* L, bool nvfp4 = false) {
   if (M < 1 || N < 1 || K < 32 || K % 32 != 0 || N % 8 != 0) return false;
   if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return false;
   if ((M + 127) / 128 > 65535) return false;
   L->k_stages = static_cast<int>((K + 255) / 256);
-  L->kgroups = 2 * L->k_stages;
+  L->kgroups = (nvfp4 ? 4 : 2) * L->k_stages;
   L->tiles_m = static_cast<int>((M + 127) / 128);
   L->tiles_n128 = 2 * static_cast<int>((N + 255) / 256);
   size_t off = kAlign;
@@ -238,21 +238,26 @@ size_t mxattn_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   return gemm_layout(M, N, K, &L) ? L.total : 0;
 }
 
-mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
-                          const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
-                          void* workspace, size_t workspace_bytes, void* stream) {
+size_t mxattn_gemm_nvfp4_workspace_size(int64_t M, int64_t N, int64_t K) {
+  GemmLayout L;
+  return gemm_layout(M, N, K, &L, true) ? L.total : 0;
+}
+
+static mxattn_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                               const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                               void* workspace, size_t workspace_bytes, void* stream, bool nvfp4) {
   if (!a_codes || !a_scales || !b_codes || !b_scales || !c || !workspace) return MXATTN_ERR_INVALID_ARG;
   if (out_dtype != MXATTN_OUT_F32 && out_dtype != MXATTN_OUT_BF16) return MXATTN_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1) return MXATTN_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(c, 16) || !aligned(workspace, 256))
     return MXATTN_ERR_INVALID_ARG;
   GemmLayout L;
-  if (!gemm_layout(M, N, K, &L)) return MXATTN_ERR_UNSUPPORTED;
+  if (!gemm_layout(M, N, K, &L, nvfp4)) return MXATTN_ERR_UNSUPPORTED;
   if (workspace_bytes < L.total) return MXATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
-  const uint32_t kb = static_cast<uint32_t>(K / 32);
+  const uint32_t kb = static_cast<uint32_t>(K / (nvfp4 ? 16 : 32));   // scale bytes per row
   const ScaleRepackParams reps[2] = {
       {a_scales, w + L.sfa, 1u, static_cast<uint32_t>(L.tiles_m), static_cast<uint32_t>(M), kb, 0,
        static_cast<uint32_t>(L.kgroups)},
@@ -284,8 +289,43 @@ mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
   p.k_stages = L.k_stages;
   p.kgroups = L.kgroups;
   p.out_bf16 = (out_dtype == MXATTN_OUT_BF16) ? 1 : 0;
+  p.nvfp4 = nvfp4 ? 1 : 0;
   p.status = reinterpret_cast<unsigned int*>(w);
   return launch_gemm(ta, tb, tc, p, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+mxattn_status mxattn_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                          const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_impl(a_codes, a_scales, b_codes, b_scales, c, M, N, K, out_dtype, workspace, workspace_bytes, stream,
+                   false);
+}
+
+mxattn_status mxattn_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                                const uint8_t* b_scales, void* c, int64_t M, int64_t N, int64_t K, int out_dtype,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_impl(a_codes, a_scales, b_codes, b_scales, c, M, N, K, out_dtype, workspace, workspace_bytes, stream,
+                   true);
+}
+
+mxattn_status mxattn_quantize_nvfp4(const void* x, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
+                                    void* stream) {
+  if (rows < 0 || cols < 0) return MXATTN_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return MXATTN_OK;
+  if (!x || !codes || !scales) return MXATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(codes, 8)) return MXATTN_ERR_INVALID_ARG;
+  if (rows >= (1ll << 31) || cols >= (1ll << 31) || static_cast<uint64_t>(rows) * ((cols + 15) / 16) >= (1ull << 40))
+    return MXATTN_ERR_UNSUPPORTED;
+  NvQuantParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.heads = 1;
+  p.rows = static_cast<uint32_t>(rows);
+  p.cols = static_cast<uint32_t>(cols);
+  p.codes = codes;
+  p.scales = scales;
+  p.vec_ok = (aligned(x, 16) && cols % 8 == 0) ? 1 : 0;
+  return launch_quantize_rows_nvfp4(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MXATTN_OK
+                                                                                          : MXATTN_ERR_CUDA;
 }
 
 

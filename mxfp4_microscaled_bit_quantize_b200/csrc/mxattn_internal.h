@@ -40,6 +40,17 @@ struct ColQuantParams {
 cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream);
 cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
 
+// NVFP4 (blocks of 16, E4M3 scales) along the contiguous axis: codes [heads*rows][ceil(cols/16)*8],
+// scales [heads*rows][ceil(cols/16)].
+struct NvQuantParams {
+  const __nv_bfloat16* x;
+  uint32_t heads, rows, cols;
+  uint8_t* codes;
+  uint8_t* scales;
+  int vec_ok;                                  // cols % 8 == 0 and x 16-byte aligned
+};
+cudaError_t launch_quantize_rows_nvfp4(const NvQuantParams& p, cudaStream_t stream);
+
 // Row-major scale bytes -> 512-byte MMA atoms [heads][tiles][512], zero where the source has no
 // element. transposed = 0: src [heads][rows][kb], atom t holds rows 128t.. and blocks 0..3;
 // transposed = 1 (V^T): src [heads][rows = channels][kb = key blocks], atom t holds channels
@@ -81,8 +92,9 @@ struct GemmParams {
   void* c;                 // [M, N] fp32 or bf16, row-major
   int M, N, K;
   int k_stages;            // ceil(K / 256)
-  int kgroups;             // 2 * k_stages (atoms per row tile, zero-padded past K)
+  int kgroups;             // atoms per row tile (zero-padded past K): 2 * k_stages, NVFP4 4 * k_stages
   int out_bf16;
+  int nvfp4;               // 0: MXFP4 (blocks of 32, UE8M0); 1: NVFP4 (blocks of 16, UE4M3)
   unsigned int* status;
 };
 

@@ -175,6 +175,52 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(ColQuantParams p) {
   }
 }
 
+// NVFP4 (comparison format): blocks of 16 along the contiguous axis, scale s = E4M3(amax / 6),
+// elements x / s on the E2M1 grid; both quotients are correctly rounded fp32 divisions, so the
+// grid decisions are taken on the same fp32 values the oracle takes them on. One thread per block.
+__global__ void __launch_bounds__(256) quantize_rows_nvfp4_kernel(const NvQuantParams p) {
+  const uint32_t nb = (p.cols + 15u) / 16u;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * p.rows * nb;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint64_t row = i / nb;
+    const uint32_t blk = static_cast<uint32_t>(i - row * nb);
+    const uint32_t c0 = blk * 16u;
+    const __nv_bfloat16* src = p.x + row * p.cols + c0;
+    float v[16];
+    if (p.vec_ok && c0 + 16u <= p.cols) {
+      const uint4 r0 = ld_stream_u4(src), r1 = ld_stream_u4(src + 8);
+      bf16x8_to_f32(r0, v);
+      bf16x8_to_f32(r1, v + 8);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = (c0 + k < p.cols) ? __bfloat162float(src[k]) : 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
+    const uint32_t byte = e4m3_byte(__fdiv_rn(amax, 6.0f));
+    const float s = e4m3_value(byte);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = (s > 0.f) ? __fdiv_rn(v[k], s) : 0.f;
+    const uint2 codes = make_uint2(cvt_e2m1x8(v), cvt_e2m1x8(v + 8));
+    *reinterpret_cast<uint2*>(p.codes + row * (nb * 8u) + blk * 8u) = codes;
+    p.scales[row * nb + blk] = static_cast<uint8_t>(byte);
+  }
+}
+
+cudaError_t launch_quantize_rows_nvfp4(const NvQuantParams& p, cudaStream_t stream) {
+  const uint64_t total = static_cast<uint64_t>(p.heads) * p.rows * ((p.cols + 15u) / 16u);
+  if (total == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t want = (total + 255) / 256;
+  const uint64_t cap = static_cast<uint64_t>(sms) * 8;
+  quantize_rows_nvfp4_kernel<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 // One thread per atom byte: invert atom_offset to find the (row, block) it holds.
 __global__ void __launch_bounds__(256) repack_scales_kernel(const ScaleRepackParams p) {
   const uint32_t kgroups = p.kgroups ? p.kgroups : 1u;

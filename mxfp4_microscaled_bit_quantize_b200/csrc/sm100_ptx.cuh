@@ -194,6 +194,19 @@ __device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// NVFP4 form: E2M1 operands, UE4M3 scales, one scale per 16 elements along K (four per row per
+// K = 64 instruction, one TMEM word), M = 128.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -253,6 +266,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 // Instruction descriptor of a dense block-scaled MMA, kind::mxf4: E2M1 A and B, both
 // K-major, UE8M0 scales, M = 128, N given; sf ids pick the scale byte pair for this K step.
+// Instruction descriptor of the NVFP4 form: E2M1 A and B, K-major, UE4M3 scales (bit 23 clear),
+// M = 128, N given.
+__host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t n) {
+  return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, uint32_t a_sf_id, uint32_t b_sf_id) {
   return (b_sf_id << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) |
          (a_sf_id << 29);
@@ -277,6 +296,20 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
       : "=r"(out)
       : "f"(hi), "f"(lo));
   return out & 0xFFu;
+}
+
+// Non-negative fp32 -> unsigned FP8 E4M3 byte, round to nearest-even, saturating at 448 (the
+// hardware conversion; the first source operand lands in the upper byte of the pair).
+__device__ __forceinline__ uint32_t e4m3_byte(float v) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  return static_cast<uint32_t>(out) & 0xFFu;
+}
+
+// Value of a non-negative finite E4M3 byte (bias 7, 3 mantissa bits), exactly.
+__device__ __forceinline__ float e4m3_value(uint32_t byte) {
+  const uint32_t e = (byte >> 3) & 0xFu, m = byte & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;   // m * 2^-9
 }
 
 // Eight fp32 values -> four bytes of codes packed into one word, element 0 in the low nibble.

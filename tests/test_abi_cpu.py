@@ -149,6 +149,22 @@ def test_gemm_workspace_and_argument_checks(lib):
     assert call(wb=good - 1) == WORKSPACE
 
 
+def test_nvfp4_argument_checks(lib):
+    q = lib.mxattn_quantize_nvfp4
+    assert q(None, 0, 16, None, None, None) == OK                   # empty: no-op
+    assert q(None, 4, 16, FAKE, FAKE, None) == INVALID
+    assert q(FAKE + 1, 4, 16, FAKE, FAKE, None) == INVALID           # misaligned x
+    assert q(FAKE, 4, 16, FAKE + 4, FAKE, None) == INVALID           # misaligned codes
+    ws = lib.mxattn_gemm_nvfp4_workspace_size
+    assert ws(4, 12, 64) == 0 and ws(4, 8, 48) == 0
+    assert ws(300, 520, 992) > lib.mxattn_gemm_workspace_size(300, 520, 992)   # twice the scale atoms
+    g = lib.mxattn_gemm_nvfp4
+    good = ws(256, 256, 512)
+    assert g(None, FAKE, FAKE, FAKE, FAKE, 256, 256, 512, 0, FAKE, good, None) == INVALID
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 256, 250, 512, 0, FAKE, good, None) == UNSUPPORTED
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 256, 256, 512, 0, FAKE, good - 1, None) == WORKSPACE
+
+
 def test_debug_argument_checks(lib):
     good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)
     r = lib.mxattn_forward_debug(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 1, 1, 0, FAKE, good, None,
