@@ -293,6 +293,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     gb = torch.randn((gn, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(6))
     g_ops = (*api.mxattn_quantize(ga.bfloat16(), False, api.SCALE_UOS),
              *api.mxattn_quantize((gb * 0.05).bfloat16(), False, api.SCALE_UOS))
+    nv_ops = (*api.mxattn_quantize_nvfp4(ga.bfloat16()), *api.mxattn_quantize_nvfp4((gb * 0.05).bfloat16()))
     del ga, gb
     g_ws = api.gemm_workspace(gm, gn, gk, dev)
     g_out = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
@@ -309,7 +310,17 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     if api.mxattn_check_status(g_ws) != 0:
         raise RuntimeError("device pipeline timeout in the GEMM")
     gemm_ms = g_start.elapsed_time(g_stop) / g_iters
-    del g_ops, g_ws, g_out
+    # the NVFP4 comparison format on the same shape (blocks of 16, E4M3 scales)
+    for _ in range(3):
+        api.mxattn_gemm_nvfp4(*nv_ops, gk, out_dtype=torch.bfloat16, out=g_out)
+    barrier()
+    g_start.record(stream)
+    for _ in range(g_iters):
+        api.mxattn_gemm_nvfp4(*nv_ops, gk, out_dtype=torch.bfloat16, out=g_out)
+    g_stop.record(stream)
+    barrier()
+    gemm_nv_ms = g_start.elapsed_time(g_stop) / g_iters
+    del g_ops, nv_ops, g_ws, g_out
 
     # standalone quantizer on its own workload (65536 x 1024 bf16), two buffer sets > L2
     xq = [synthetic.quant_input().to(dev) for _ in range(2)]
@@ -328,8 +339,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
-    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms = reduce_max_over_ranks(
-        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms], world, dev)
+    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms = reduce_max_over_ranks(
+        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms], world, dev)
     if rank != 0:
         return
 
@@ -373,6 +384,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
                  "tflops": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12,
                  "frac": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12 / fp4_peak,
+                 "nvfp4": {"ms": gemm_nv_ms, "tflops": 2.0 * gm * gn * gk / (gemm_nv_ms * 1e-3) / 1e12,
+                           "frac": 2.0 * gm * gn * gk / (gemm_nv_ms * 1e-3) / 1e12 / fp4_peak},
                  "capture_traffic": {"workload": "2048x16384x8192 (M reduced for the ncu capture)",
                                      "dram_bytes": profile_traffic("mxgemm_2048x16384x8192.json",
                                                                    sources_hash(GEMM_SOURCES))}},
