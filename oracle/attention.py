@@ -42,12 +42,16 @@ Readings taken where the pages are silent (each also listed in the design notes)
   its block amax, scale exponent and code are chosen. Everything else stays fp64.
 * Keys >= N and (causal) keys > i are masked: p = 0, code +0; an all-masked 32-key
   block gets scale byte 0x00.
+* mode = 2 (nvfp4.SCALE_NVFP4) is the NVFP4 comparison format of oracle/nvfp4.py for all four
+  operands: blocks of 16 with E4M3 scales; P~ blocks are 16 keys, each decision again taken on
+  the fp32-rounded P~ (scale byte from fp32(amax / 6), element from fp32(p / s)).
 """
 from __future__ import annotations
 
 import numpy as np
 
 from . import mxfp4 as mx
+from . import nvfp4 as nv
 
 KV_TILE = 64          # the library's documented tile width (MXATTN_KV_TILE)
 
@@ -59,6 +63,14 @@ def dequantized_qkv(q, k, v, mode: int):
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     N, d = q.shape[-2], q.shape[-1]
+    if mode == nv.SCALE_NVFP4:
+        qc, qs = nv.quantize_rows(q)
+        kc, ks = nv.quantize_rows(k)
+        vc, vs = nv.quantize_rows(np.swapaxes(v, -1, -2))  # [.., d, ceil(N/16)*8], [.., d, ceil(N/16)]
+        qd = nv.dequantize_rows(qc, qs, d)
+        kd = nv.dequantize_rows(kc, ks, d)
+        vd = np.swapaxes(nv.dequantize_rows(vc, vs, N), -1, -2)
+        return (qd, kd, vd), dict(qc=qc, qs=qs, kc=kc, ks=ks, vc=vc, vs=vs)
     qc, qs = mx.quantize_rows(q, mode)
     kc, ks = mx.quantize_rows(k, mode)
     vc, vs = mx.quantize_transposed(v, mode)            # [.., d, Npad/2], [.., d, Npad/32]
@@ -68,10 +80,20 @@ def dequantized_qkv(q, k, v, mode: int):
     return (qd, kd, vd), dict(qc=qc, qs=qs, kc=kc, ks=ks, vc=vc, vs=vs)
 
 
+def block_size(mode: int) -> int:
+    return nv.BLOCK if mode == nv.SCALE_NVFP4 else mx.BLOCK
+
+
 def _quantize_p(p32: np.ndarray, mode: int):
-    """PNQ step: MXFP4 round trip of P~ rows along keys (blocks of 32 absolute keys).
-    p32: [R, T] with T a multiple of 32. Returns (dequantized fp64, codes, scale bytes)."""
+    """PNQ step: round trip of P~ rows along keys in the mode's format (MXFP4: blocks of 32
+    absolute keys; NVFP4: blocks of 16). p32: [R, T] with T a multiple of the block.
+    Returns (dequantized fp64, codes, scale bytes)."""
     R, T = p32.shape
+    if mode == nv.SCALE_NVFP4:
+        pb = p32.astype(np.float64).reshape(R, T // nv.BLOCK, nv.BLOCK)
+        codes, sbytes = nv.quantize_blocks(pb)
+        deq = mx.e2m1_decode(codes) * nv.e4m3_decode(sbytes)[..., None]
+        return deq.reshape(R, T), codes.reshape(R, T), sbytes
     pb = p32.astype(np.float64).reshape(R, T // mx.BLOCK, mx.BLOCK)
     codes, e = mx.quantize_blocks(pb, mode)
     deq = np.ldexp(mx.e2m1_decode(codes), e[..., None]).reshape(R, T)
@@ -91,6 +113,7 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
     qd_rows = np.asarray(qd_rows, dtype=np.float64)
     row_idx = np.asarray(row_idx, dtype=np.int64)
     N, d = kd.shape
+    blk = block_size(mode)
     assert kv_tile % mx.BLOCK == 0
     R = qd_rows.shape[0]
     sigma = 1.0 / np.sqrt(d)
@@ -101,9 +124,9 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
     if record_p:
         npad = n_tiles * kv_tile
         rec_codes = np.zeros((R, npad), dtype=np.uint8)
-        rec_scales = np.zeros((R, npad // mx.BLOCK), dtype=np.uint8)
+        rec_scales = np.zeros((R, npad // blk), dtype=np.uint8)
         rec_y = np.zeros((R, npad))
-        rec_amax = np.zeros((R, npad // mx.BLOCK))
+        rec_amax = np.zeros((R, npad // blk))
     for t in range(n_tiles):
         j0 = t * kv_tile
         keys = np.arange(j0, j0 + kv_tile)
@@ -127,13 +150,19 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
             denom = qv if pnq else p32.astype(np.float64)
             if record_p:
                 rec_codes[:, j0:j0 + kv_tile] = codes
-                nb0 = j0 // mx.BLOCK
-                rec_scales[:, nb0:nb0 + kv_tile // mx.BLOCK] = sbytes
-                e = sbytes.astype(np.int64) - mx.E8M0_BIAS
-                rec_y[:, j0:j0 + kv_tile] = np.ldexp(
-                    p32.astype(np.float64).reshape(R, -1, mx.BLOCK), -e[..., None]).reshape(R, -1)
-                rec_amax[:, nb0:nb0 + kv_tile // mx.BLOCK] = (
-                    p32.astype(np.float64).reshape(R, -1, mx.BLOCK).max(axis=-1))
+                nb0 = j0 // blk
+                rec_scales[:, nb0:nb0 + kv_tile // blk] = sbytes
+                pbk = p32.astype(np.float64).reshape(R, -1, blk)
+                if mode == nv.SCALE_NVFP4:   # y = fp32(p / s), amax recorded as fp32(amax / 6)
+                    s_ = nv.e4m3_decode(sbytes)[..., None]
+                    with np.errstate(divide="ignore", invalid="ignore"):
+                        yv = np.where(s_ > 0, (pbk / s_).astype(np.float32), 0.0)
+                    rec_y[:, j0:j0 + kv_tile] = yv.reshape(R, -1)
+                    rec_amax[:, nb0:nb0 + kv_tile // blk] = (pbk.max(axis=-1) / 6.0).astype(np.float32)
+                else:
+                    e = sbytes.astype(np.int64) - mx.E8M0_BIAS
+                    rec_y[:, j0:j0 + kv_tile] = np.ldexp(pbk, -e[..., None]).reshape(R, -1)
+                    rec_amax[:, nb0:nb0 + kv_tile // blk] = pbk.max(axis=-1)
         else:
             qv = p
             denom = p

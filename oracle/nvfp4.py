@@ -24,6 +24,7 @@ import numpy as np
 from . import mxfp4 as mx
 
 BLOCK = 16
+SCALE_NVFP4 = 2          # the attention oracle's mode number for this format (MXFP4: OCP 0, UOS 1)
 E4M3_MAX = 448.0
 E4M3_NAN = 0x7F
 

@@ -16,6 +16,7 @@ from __future__ import annotations
 import numpy as np
 
 from oracle import mxfp4 as mx
+from oracle import nvfp4 as nv
 
 OUT_MAX_ABS = 5e-3
 OUT_REL_FRO = 1e-3
@@ -29,9 +30,16 @@ def near_midpoint(y: np.ndarray) -> np.ndarray:
     return (np.abs(a - MIDPOINTS) <= TIE_REL * MIDPOINTS).any(axis=-1)
 
 
+_E4M3_VALS = nv.e4m3_decode(np.arange(0x7F))
+_E4M3_MIDS = (_E4M3_VALS[1:] + _E4M3_VALS[:-1]) / 2
+
+
 def near_scale_boundary(amax: np.ndarray, mode: int) -> np.ndarray:
-    """amax within TIE_REL of a power of two (both rules) or of 1.8125 * 2^k (UOS)."""
+    """MXFP4: amax within TIE_REL of a power of two (both rules) or of 1.8125 * 2^k (UOS).
+    NVFP4: the recorded fp32(amax / 6) within TIE_REL of an E4M3 rounding midpoint."""
     a = np.asarray(amax, dtype=np.float64)
+    if mode == nv.SCALE_NVFP4:
+        return (np.abs(a[..., None] - _E4M3_MIDS) <= TIE_REL * _E4M3_MIDS).any(axis=-1)
     out = np.zeros(a.shape, dtype=bool)
     pos = a > 0
     frac, ex = np.frexp(a[pos])            # a = frac * 2^ex, frac in [0.5, 1)
@@ -46,16 +54,17 @@ def near_scale_boundary(amax: np.ndarray, mode: int) -> np.ndarray:
 def classify_p_mismatches(gpu_codes, gpu_scales, rec, mode, n_valid):
     """Compare GPU P~ dumps with the oracle's record for the same rows.
 
-    gpu_codes [R, Npad/2] packed, gpu_scales [R, Npad/32]; rec from attention_rows(record_p=True).
-    Returns dict(rate, n, mismatches, unexplained, scale_mismatch_blocks).
+    gpu_codes [R, Npad/2] packed, gpu_scales [R, Npad/blk] (blk = 32, or 16 for NVFP4); rec from
+    attention_rows(record_p=True). Returns dict(rate, n, mismatches, unexplained, scale_mismatch_blocks).
     """
+    bs = nv.BLOCK if mode == nv.SCALE_NVFP4 else mx.BLOCK
     g = mx.unpack_nibbles(np.asarray(gpu_codes))[:, :n_valid]
     o = rec["codes"][:, :n_valid]
-    nb_valid = -(-n_valid // 32)
+    nb_valid = -(-n_valid // bs)
     gs = np.asarray(gpu_scales)[:, :nb_valid]
     os_ = rec["scales"][:, :nb_valid]
     code_mis = g != o
-    blk = np.repeat(np.arange(nb_valid), 32)[:n_valid]
+    blk = np.repeat(np.arange(nb_valid), bs)[:n_valid]
     scale_mis_blk = gs != os_
     explained_blk = near_scale_boundary(rec["amax"][:, :nb_valid], mode)
     explained = near_midpoint(rec["y"][:, :n_valid]) | explained_blk[:, blk]

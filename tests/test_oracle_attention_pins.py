@@ -45,19 +45,24 @@ def test_loop_equals_softmax_without_quantization(causal, N):
         assert np.max(np.abs(got - ref)) <= 1e-12
 
 
-@pytest.mark.parametrize("mode", [mx.SCALE_OCP, mx.SCALE_UOS])
+@pytest.mark.parametrize("mode", [mx.SCALE_OCP, mx.SCALE_UOS, 2])
 def test_pnq_preserves_normalisation(mode):
     rng = np.random.default_rng(3)
     N, d = 300, 64
     q = _bf16(rng.standard_normal((1, 2, N, d)) * 3.0)    # sharp rows
     k = _bf16(rng.standard_normal((1, 2, N, d)) * 3.0)
-    v = np.ones((1, 2, N, d))                              # dq(V) = 1 exactly
+    v = np.ones((1, 2, N, d))
+    # every V entry dequantizes to one constant: 1 in MXFP4 (code 1.0, scale 2^-2 ... exact), and
+    # 6 * E4M3(1/6) = 1.03125 in NVFP4; a normalised softmax must return exactly that constant
+    (_, _, vd), _ = oa.dequantized_qkv(q[0, 0], k[0, 0], v[0, 0], mode)
+    vconst = vd[0, 0]
+    assert np.all(vd == vconst)
     out_pnq = oa.mxattention(q, k, v, causal=False, mode=mode, pnq=True)
     out_conv = oa.mxattention(q, k, v, causal=False, mode=mode, pnq=False)
-    assert np.max(np.abs(out_pnq - 1.0)) <= 1e-12
-    assert np.max(np.abs(out_conv - 1.0)) > 1e-3          # numerator/denominator mismatch
+    assert np.max(np.abs(out_pnq - vconst)) <= 1e-12
+    assert np.max(np.abs(out_conv - vconst)) > 1e-3       # numerator/denominator mismatch
     out_causal = oa.mxattention(q, k, v, causal=True, mode=mode, pnq=True)
-    assert np.max(np.abs(out_causal - 1.0)) <= 1e-12
+    assert np.max(np.abs(out_causal - vconst)) <= 1e-12
 
 
 def test_uniform_scores_by_hand():
@@ -153,3 +158,24 @@ def test_softmax_stage_error_ordering():
     e_best = mx.rel_frobenius(_p_only(q, k, v2, mx.SCALE_UOS, True), ref2)
     e_base = mx.rel_frobenius(_p_only(q, k, v2, mx.SCALE_OCP, False), ref2)
     assert e_best * 1.5 < e_base, (e_best, e_base)
+
+
+def test_uniform_scores_by_hand_nvfp4():
+    """NVFP4 mode: every P~ = 1 -> fp32(1/6) rounds to the E4M3 scale 1.375 * 2^-3 = 0.171875
+    (byte 0x23: exponent field 4, mantissa 3), 1 / 0.171875 = 5.82 rounds to the top E2M1 value 6
+    (code 7); all weights equal, so the output is the mean of the dequantized V rows."""
+    from oracle import nvfp4 as nv
+    N, d = 80, 64
+    q = np.full((1, 1, N, d), 0.5)
+    k = np.full((1, 1, N, d), 0.25)
+    rng = np.random.default_rng(10)
+    v = _bf16(rng.standard_normal((1, 1, N, d)))
+    (qd, kd, vd), _ = oa.dequantized_qkv(q[0, 0], k[0, 0], v[0, 0], nv.SCALE_NVFP4)
+    out, rec = oa.attention_rows(qd, np.arange(N), kd, vd, causal=False, mode=nv.SCALE_NVFP4,
+                                 pnq=True, record_p=True)
+    valid = np.arange(rec["codes"].shape[1]) < N
+    assert np.all(rec["codes"][:, valid] == 7)
+    nb = N // 16
+    assert np.all(rec["scales"][:, :nb] == 0x23)
+    assert np.all(rec["scales"][:, nb:] == 0)              # all-masked padded blocks
+    assert np.max(np.abs(out - vd.mean(axis=0)[None, :])) <= 1e-14
