@@ -13,6 +13,9 @@
  *       MXATTN_SCALE_OCP: e = floor(log2 amax) - 2        (the OCP MX v1.0 rule)
  *       MXATTN_SCALE_UOS: smallest e with amax / 2^e <= 7.25 (Universal Optimal Scaling)
  *     An all-zero block gets scale byte 0 and all-zero codes.
+ *       MXATTN_SCALE_NVFP4: the NVFP4 comparison format for Q, K, V and P~ instead (blocks of
+ *       16 with an E4M3 scale RNE(amax / 6); see mxattn_quantize_nvfp4); mxattn_forward and its
+ *       prepare / attend / debug forms only.
  *   - Attention: Q, K quantized along the head dimension, V along keys; S = Q K^T as a
  *     block-scaled FP4 contraction; FlashAttention online softmax over key tiles of
  *     MXATTN_KV_TILE keys in increasing key order (running max, history rescale, fp32
@@ -46,7 +49,7 @@
 extern "C" {
 #endif
 
-typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1 } mxattn_scale_mode;
+typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1, MXATTN_SCALE_NVFP4 = 2 } mxattn_scale_mode;
 
 /* Keys per tile of the online softmax. P~ is quantized with the running max in force at each
  * tile, so the tile width is part of the result (a CPU reference must use the same width). */
@@ -112,7 +115,8 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* 
  *   vtc : codes  [B, Hkv, d, ceil(N/32)*16]  (mxattn_quantize of v with transpose = 1: blocks of
  *         32 keys, keys past N encoded as zero), 16-byte aligned
  *   vts : scales [B, Hkv, d, ceil(N/32)]
- *   p_scale_mode: the scale rule for P~ (the caller chose the rule of Q, K, V when quantizing).
+ *   p_scale_mode: the scale rule for P~ (the caller chose the rule of Q, K, V when quantizing);
+ *   MXATTN_SCALE_OCP or MXATTN_SCALE_UOS (MXATTN_SCALE_NVFP4 -> MXATTN_ERR_UNSUPPORTED).
  * All other arguments as mxattn_forward; the workspace (mxattn_forward_workspace_size bytes)
  * receives the scales in the tensor-core layout and the status word; the codes are read in place
  * and must stay unchanged until the call has completed on the stream. Errors: null or misaligned
@@ -190,7 +194,8 @@ mxattn_status mxattn_forward_attend(void* out, int B, int Hq, int Hkv, int N, in
 /*
  * mxattn_forward_debug -- mxattn_forward that also dumps the quantized P~ operand of query
  * rows [r0, r1) of head dbg_bh (= b * Hq + h): p_codes [r1-r0][Npad/2] packed codes and
- * p_scales [r1-r0][Npad/32] scale bytes in absolute key order, Npad = ceil(N/128)*128
+ * p_scales [r1-r0][Npad/32] scale bytes in absolute key order (Npad/16 for MXATTN_SCALE_NVFP4),
+ * Npad = ceil(N/128)*128
  * (device memory). Meant for parity tests on small shapes.
  */
 mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, void* out, int B, int Hq,

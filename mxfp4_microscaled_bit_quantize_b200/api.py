@@ -10,7 +10,7 @@ import torch
 
 from . import _lib
 
-SCALE_OCP, SCALE_UOS = 0, 1
+SCALE_OCP, SCALE_UOS, SCALE_NVFP4 = 0, 1, 2
 OUT_F32, OUT_BF16 = 0, 1
 KV_TILE = 64          # keys per online-softmax tile (MXATTN_KV_TILE)
 NPAD_ALIGN = 128      # the workspace pads N to a multiple of this
@@ -236,14 +236,14 @@ def mxattn_forward_debug(q, k, v, dbg_bh: int, r0: int, r1: int, causal: bool = 
                          scale_mode: int = SCALE_UOS, pnq: bool = True, out_dtype=torch.float32,
                          workspace: torch.Tensor | None = None):
     """mxattn_forward plus the quantized P~ of rows [r0, r1) of head dbg_bh (= b*Hq + h):
-    returns (out, p_codes [r1-r0, Npad/2], p_scales [r1-r0, Npad/32])."""
+    returns (out, p_codes [r1-r0, Npad/2], p_scales [r1-r0, Npad/32], or Npad/16 for NVFP4)."""
     B, Hq, Hkv, N, d = _shapes(q, k, v)
     out, od = _out(q, out_dtype, None)
     if workspace is None:
         workspace = alloc_workspace(B, Hq, Hkv, N, d, q.device)
     npd = npad(N)
     pc = torch.zeros((r1 - r0, npd // 2), dtype=torch.uint8, device=q.device)
-    ps = torch.zeros((r1 - r0, npd // 32), dtype=torch.uint8, device=q.device)
+    ps = torch.zeros((r1 - r0, npd // (16 if scale_mode == SCALE_NVFP4 else 32)), dtype=torch.uint8, device=q.device)
     st = _lib.load().mxattn_forward_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
                                           Hkv, N, d, int(bool(causal)), int(scale_mode), int(bool(pnq)), od,
                                           workspace.data_ptr(), workspace.numel(), _stream(q.device),

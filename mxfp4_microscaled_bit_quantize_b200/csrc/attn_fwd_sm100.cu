@@ -44,13 +44,15 @@ constexpr int kBN = kKvTile;      // keys per KV tile (64)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 64, kColL = 192;
-constexpr uint32_t kColSfQ = 208, kColSfK = 212, kColSf1 = 216;
+// Q and K scale atoms: one per 64 (NVFP4) or 128 (MXFP4) contraction elements, 4 columns each.
+constexpr uint32_t kColSfQ = 208, kColSfK = 216, kColSf1 = 224;
 // P~ scale atoms alternate between two column sets by tile parity, V scale atoms (one per pair of
 // 64-key tiles) by pair parity: tcgen05.cp into columns an earlier MMA still reads is not ordered
 // behind that MMA, and the product of tile j may still run when the scales of tile j+1 are
 // copied. The set written for tile j+1 was last read by a product no later than that of tile
 // j-1, which the softmax has seen complete before it hands over tile j+1.
-constexpr uint32_t kColSfV = 220, kColSfP = 228;   // + 4 * set
+// NVFP4 gives every 64-key tile its own V atom, which then alternates by tile parity.
+constexpr uint32_t kColSfV = 228, kColSfP = 236;   // + 4 * set
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
 constexpr int kPRowBytes = kBN / 2;                  // 32 bytes of codes per P~ row
 constexpr size_t kMinSmem = 80 * 1024;               // at most two CTAs per SM (TMEM halves)
@@ -75,8 +77,8 @@ struct __align__(1024) Smem {
   uint8_t v[Cfg<D>::kStages][Cfg<D>::kVTileBytes];
   uint8_t p[2][kBM * kPRowBytes];         // P~ codes, double-buffered by tile parity
   uint8_t ones[kOnesRows * kPRowBytes];
-  uint8_t qsf[512];
-  uint8_t ksf[Cfg<D>::kStages][512];
+  uint8_t qsf[1024];                      // MXFP4: one atom; NVFP4: D / 64 atoms
+  uint8_t ksf[Cfg<D>::kStages][1024];
   uint8_t vsf[Cfg<D>::kStages][512];
   uint8_t psf[2][512];
   uint8_t onesf[512];
@@ -137,12 +139,29 @@ __device__ __forceinline__ float block_max32(const float* v) {
   return fmaxf(fmax3(a0, a1, a2), a3);
 }
 
-template <int D, bool PNQ, bool DBG>
+// max over 16 consecutive values
+__device__ __forceinline__ float block_max16(const float* v) {
+  const float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]), a2 = fmax3(v[6], v[7], v[8]);
+  const float a3 = fmax3(v[9], v[10], v[11]), a4 = fmax3(v[12], v[13], v[14]);
+  return fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]));
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// NV = false: MXFP4 (blocks of 32, UE8M0, OCP or UOS exponent). NV = true: the NVFP4 comparison
+// format for Q, K, V and P~ (blocks of 16, E4M3 scale = RNE(amax / 6)).
+template <int D, bool PNQ, bool DBG, bool NV>
 __global__ void __launch_bounds__(kThreads, 2)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
+  constexpr int kQKAtoms = NV ? D / 64 : 1;            // scale atoms per 128 Q or K rows
+  constexpr uint32_t kQKSfBytes = kQKAtoms * 512;
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& s = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -198,9 +217,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(&s.bar_q, C::kQTileBytes + 512);
+      mbar_arrive_expect_tx(&s.bar_q, C::kQTileBytes + kQKSfBytes);
       tma_load_2d(s.q, &tmQ, &s.bar_q, 0, bh_q * p.rows_per_head + qt * kBM);
-      bulk_load(s.qsf, p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt) * 512, 512, &s.bar_q);
+      bulk_load(s.qsf, p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt) * kQKSfBytes, kQKSfBytes, &s.bar_q);
     }
     __syncwarp();
     int issued = 0;
@@ -212,15 +231,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (leader) {
-        // scale atoms cover 128 keys: tiles 2t and 2t+1 share atom t, loaded with the even tile
+        // K scale atoms cover 128 keys: tiles 2t and 2t+1 share them, loaded with the even tile;
+        // V atoms likewise for MXFP4, one per 64-key tile for NVFP4
         const bool atoms = (j & 1) == 0;
-        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + (atoms ? 1024 : 0));
+        const bool v_atom = NV || atoms;
+        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + (atoms ? kQKSfBytes : 0) +
+                                                      (v_atom ? 512 : 0));
         tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.rows_per_head + j * kBN);
         tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
-        if (atoms) {
-          const size_t atom = (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * 512;
-          bulk_load(s.ksf[st], p.ksf + atom, 512, &s.bar_kv_full[st]);
-          bulk_load(s.vsf[st], p.vsf + atom, 512, &s.bar_kv_full[st]);
+        if (atoms)
+          bulk_load(s.ksf[st], p.ksf + (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * kQKSfBytes, kQKSfBytes,
+                    &s.bar_kv_full[st]);
+        if (v_atom) {
+          const size_t v_at = NV ? static_cast<size_t>(bh_kv) * (p.Npad / kBN) + j
+                                 : static_cast<size_t>(bh_kv) * n_qt + (j >> 1);
+          bulk_load(s.vsf[st], p.vsf + v_at * 512, 512, &s.bar_kv_full[st]);
         }
       }
       __syncwarp();
@@ -244,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
       for (int i = lane; i < kOnesRows * kPRowBytes / 4; i += 32) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
       uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
-      for (int i = lane; i < 512 / 4; i += 32) sw[i] = 0x7F7F7F7Fu;
+      for (int i = lane; i < 512 / 4; i += 32) sw[i] = NV ? 0x38383838u : 0x7F7F7F7Fu;   // E4M3 / E8M0 1.0
       fence_proxy_async_smem();
     }
     __syncwarp();
@@ -253,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok) {
       tc_fence_after();
       if (leader) {
-        tc_cp_sf(tmem + kColSfQ, sf_desc(s.qsf));
+#pragma unroll
+        for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfQ + 4 * a, sf_desc(s.qsf + a * 512));
         if (PNQ) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
       }
       __syncwarp();
@@ -272,13 +298,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
       const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
       if (leader) {
-        // the even tile brings the K atom of the pair; S of the previous pair has completed
-        if ((j & 1) == 0) tc_cp_sf(tmem + kColSfK, sf_desc(s.ksf[st]));
+        // the even tile brings the K atoms of the pair; S of the previous pair has completed
+        if ((j & 1) == 0) {
+#pragma unroll
+          for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfK + 4 * a, sf_desc(s.ksf[st] + a * 512));
+        }
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
           const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
           const uint64_t bd = smem_desc(ka + kk * 32, 0, C::kQKSbo, C::kQKLayout);
-          tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ, sfk, kk > 0);
+          if constexpr (NV)   // one atom (four 16-element blocks) per K = 64 step
+            tc_mma_nvf4(tmem + kColS, ad, bd, idesc_nvf4(kBN), tmem + kColSfQ + 4 * kk, sfk + 4 * kk, kk > 0);
+          else
+            tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ, sfk, kk > 0);
         }
         tc_commit(&s.bar_s_full);
       }
@@ -294,16 +326,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
       const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
       if (leader) {
-        const uint32_t sfp = tmem + kColSfP + 4 * (j & 1), sfv = tmem + kColSfV + 4 * ((j >> 1) & 1);
+        const uint32_t sfp = tmem + kColSfP + 4 * (j & 1);
+        const uint32_t sfv = tmem + kColSfV + 4 * (NV ? (j & 1) : ((j >> 1) & 1));
         tc_cp_sf(sfp, sf_desc(s.psf[j & 1]));
-        if ((j & 1) == 0) tc_cp_sf(sfv, sf_desc(s.vsf[st]));   // the V atom of the tile pair
-        // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
-        tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), sfp, sfv,
-                    j > 0 ? 1u : 0u);
-        if (PNQ) {
-          const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
-          tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), sfp, tmem + kColSf1,
-                      j > 0 ? 1u : 0u);
+        if (NV || (j & 1) == 0) tc_cp_sf(sfv, sf_desc(s.vsf[st]));   // MXFP4: the V atom of the tile pair
+        if constexpr (NV) {
+          tc_mma_nvf4(tmem + kColO, ad, bd, idesc_nvf4(D), sfp, sfv, j > 0 ? 1u : 0u);
+          if (PNQ) {
+            const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
+            tc_mma_nvf4(tmem + kColL, ad, od, idesc_nvf4(kOnesRows), sfp, tmem + kColSf1, j > 0 ? 1u : 0u);
+          }
+        } else {
+          // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
+          tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), sfp, sfv, j > 0 ? 1u : 0u);
+          if (PNQ) {
+            const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
+            tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), sfp, tmem + kColSf1,
+                        j > 0 ? 1u : 0u);
+          }
         }
         tc_commit(&s.bar_pv_done[j & 1]);
         tc_commit(&s.bar_kv_empty[st]);
@@ -366,42 +406,59 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (key >= p.N || (p.causal && key > qrow)) sv[i] = -INFINITY;
         }
       }
-      float bmax[kBN / 32];
+      // per block (32 keys for MXFP4, 16 for NVFP4): amax from the exact difference (1 for the
+      // block that holds the max), the block's scale byte, and the exponent bias nb of
+      // y = P~ / s = 2^(S c - m c - log2 s): one FFMA + one ex2 per element
+      constexpr int kPB = NV ? 16 : 32;          // keys per P~ scale block
+      constexpr int kNPB = kBN / kPB;
+      float bmax[kNPB];
 #pragma unroll
-      for (int bb = 0; bb < kBN / 32; ++bb) bmax[bb] = block_max32(sv + bb * 32);
-      const float m_new = fmaxf(m, fmaxf(bmax[0], bmax[1]));
+      for (int bb = 0; bb < kNPB; ++bb) bmax[bb] = NV ? block_max16(sv + bb * kPB) : block_max32(sv + bb * kPB);
+      float tmax = bmax[0];
+#pragma unroll
+      for (int bb = 1; bb < kNPB; ++bb) tmax = fmaxf(tmax, bmax[bb]);
+      const float m_new = fmaxf(m, tmax);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
 
-      // per 32-key block: amax from the exact difference (1 for the block that holds the max),
-      // its E8M0 byte, and the exponent bias of y = P~ / 2^e = 2^(S c - m c - e)
-      uint32_t byte[kBN / 32];
-      float nb[kBN / 32];
+      uint32_t sbytes = 0;
+      float nb[kNPB], bscale[kNPB];
 #pragma unroll
-      for (int bb = 0; bb < kBN / 32; ++bb) {
+      for (int bb = 0; bb < kNPB; ++bb) {
         const float amax = ex2_approx((bmax[bb] - m_use) * c);     // 0 for an all-masked block
-        byte[bb] = e8m0_scale_byte(amax, p.mode);
-        nb[bb] = fmaf(-m_use, c, static_cast<float>(127 - static_cast<int>(byte[bb])));
+        uint32_t byte;
+        if constexpr (NV) {
+          // s = E4M3(amax / 6) with both quotients correctly rounded. s = 0 (amax <= 6 * 2^-10):
+          // y = P~ itself (every value below the 0.25 rounding threshold, so the codes are 0 as
+          // the format wants) and the unquantized row sum still counts the block with weight 1
+          byte = e4m3_byte(__fdiv_rn(amax, 6.0f));
+          const float sb = e4m3_value(byte);
+          bscale[bb] = sb > 0.f ? sb : 1.f;
+          nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
+        } else {
+          byte = e8m0_scale_byte(amax, p.mode);
+          bscale[bb] = pow2_from_byte(byte);
+          nb[bb] = fmaf(-m_use, c, static_cast<float>(127 - static_cast<int>(byte)));
+        }
+        sbytes |= byte << (8 * bb);
       }
-      const uint32_t sbytes = byte[0] | (byte[1] << 8);
-      // y for the whole tile (one FFMA + one ex2 per element), then the E2M1 codes
       float y[kBN];
 #pragma unroll
-      for (int i = 0; i < kBN; ++i) y[i] = ex2_approx_ftz(fmaf(sv[i], c, nb[i / 32]));
+      for (int i = 0; i < kBN; ++i) y[i] = ex2_approx_ftz(fmaf(sv[i], c, nb[i / kPB]));
       uint32_t words[kBN / 8];          // 8 words = 32 bytes of codes for this row
 #pragma unroll
       for (int w = 0; w < kBN / 8; ++w) words[w] = cvt_e2m1x8(y + 8 * w);
       if (!PNQ) {   // conventional row sum of the unquantized exponentials
         float tile_sum = 0.f;
 #pragma unroll
-        for (int bb = 0; bb < kBN / 32; ++bb) {
+        for (int bb = 0; bb < kNPB; ++bb) {
           float b0 = 0.f, b1 = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            b0 += y[bb * 32 + i];
-            b1 += y[bb * 32 + i + 1];
+          for (int i = 0; i < kPB; i += 2) {
+            b0 += y[bb * kPB + i];
+            b1 += y[bb * kPB + i + 1];
           }
-          tile_sum = fmaf(b0 + b1, pow2_from_byte(byte[bb]), tile_sum);
+          tile_sum = fmaf(b0 + b1, bscale[bb], tile_sum);
         }
         l = fmaf(alpha, l, tile_sum);
       }
@@ -419,15 +476,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint4 v4 = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
         *reinterpret_cast<uint4*>(p_row + ((bb ^ swz) << 4)) = v4;
       }
-      *reinterpret_cast<uint16_t*>(s.psf[pb] + psf_off) = static_cast<uint16_t>(sbytes);
+      if constexpr (NV)
+        *reinterpret_cast<uint32_t*>(s.psf[pb] + psf_off) = sbytes;            // 4 blocks of 16 keys
+      else
+        *reinterpret_cast<uint16_t*>(s.psf[pb] + psf_off) = static_cast<uint16_t>(sbytes);
       if (DBG && dbg) {
         uint4* dc = reinterpret_cast<uint4*>(p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) +
                                              j * kPRowBytes);
 #pragma unroll
         for (int bb = 0; bb < kBN / 32; ++bb)
           dc[bb] = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
-        *reinterpret_cast<uint16_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 32) +
-                                     j * 2) = static_cast<uint16_t>(sbytes);
+        if constexpr (NV)
+          *reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 16) + j * 4) =
+              sbytes;
+        else
+          *reinterpret_cast<uint16_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 32) + j * 2) =
+              static_cast<uint16_t>(sbytes);
       }
       fence_proxy_async_smem();
 
@@ -520,26 +584,33 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D, bool PNQ, bool DBG>
+template <int D, bool PNQ, bool DBG, bool NV>
 static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ, DBG>,
+  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ, DBG, NV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * (p.Npad / kBM);
-  mxattn_fwd_kernel<D, PNQ, DBG><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PNQ, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
+}
+
+template <int D, bool NV>
+static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const AttnParams& p, cudaStream_t stream) {
+  const bool dbg = p.dbg_codes != nullptr;
+  if (p.pnq) return dbg ? launch_k<D, true, true, NV>(tmQ, tmK, tmV, p, stream)
+                        : launch_k<D, true, false, NV>(tmQ, tmK, tmV, p, stream);
+  return dbg ? launch_k<D, false, true, NV>(tmQ, tmK, tmV, p, stream)
+             : launch_k<D, false, false, NV>(tmQ, tmK, tmV, p, stream);
 }
 
 template <int D>
 static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
-  const bool dbg = p.dbg_codes != nullptr;
-  if (p.pnq) return dbg ? launch_k<D, true, true>(tmQ, tmK, tmV, p, stream)
-                        : launch_k<D, true, false>(tmQ, tmK, tmV, p, stream);
-  return dbg ? launch_k<D, false, true>(tmQ, tmK, tmV, p, stream)
-             : launch_k<D, false, false>(tmQ, tmK, tmV, p, stream);
+  return p.mode == kModeNvfp4 ? launch_f<D, true>(tmQ, tmK, tmV, p, stream)
+                              : launch_f<D, false>(tmQ, tmK, tmV, p, stream);
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,

@@ -39,11 +39,14 @@ bool ws_layout(int B, int Hq, int Hkv, int N, int d, WsLayout* L) {
     return o;
   };
   L->qc = take(static_cast<size_t>(B) * Hq * npad * (d / 2));
-  L->qs = take(static_cast<size_t>(B) * Hq * tiles * 512);
+  // scale regions sized for the larger format: NVFP4 has d / 64 atoms per 128 Q / K rows and one
+  // V atom per 64 keys (MXFP4 uses the first 512 bytes per 128 rows or keys, packed)
+  const size_t qk_atoms = (d >= 128) ? static_cast<size_t>(d / 64) : 1;
+  L->qs = take(static_cast<size_t>(B) * Hq * tiles * qk_atoms * 512);
   L->kc = take(static_cast<size_t>(B) * Hkv * npad * (d / 2));
-  L->ks = take(static_cast<size_t>(B) * Hkv * tiles * 512);
+  L->ks = take(static_cast<size_t>(B) * Hkv * tiles * qk_atoms * 512);
   L->vc = take(static_cast<size_t>(B) * Hkv * d * (npad / 2));
-  L->vs = take(static_cast<size_t>(B) * Hkv * tiles * 512);
+  L->vs = take(static_cast<size_t>(B) * Hkv * tiles * 1024);
   L->total = off;
   L->npad = static_cast<int>(npad);
   return true;
@@ -101,6 +104,35 @@ mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, i
     if (cudaMemsetAsync(w + L.qs, 0, L.kc - L.qs, st) != cudaSuccess) return MXATTN_ERR_CUDA;
     if (cudaMemsetAsync(w + L.ks, 0, L.vc - L.ks, st) != cudaSuccess) return MXATTN_ERR_CUDA;
     if (cudaMemsetAsync(w + L.vs, 0, L.total - L.vs, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  }
+  if (scale_mode == kModeNvfp4) {
+    NvQuantParams nq{};
+    nq.x = static_cast<const __nv_bfloat16*>(q);
+    nq.heads = static_cast<uint32_t>(B * Hq);
+    nq.rows = static_cast<uint32_t>(N);
+    nq.rows_pad = static_cast<uint32_t>(L.npad);
+    nq.cols = static_cast<uint32_t>(d);
+    nq.codes = w + L.qc;
+    nq.scales = w + L.qs;
+    nq.vec_ok = aligned(q, 16) ? 1 : 0;
+    nq.sf_layout = kSfAtom;
+    if (launch_quantize_rows_nvfp4(nq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    nq.x = static_cast<const __nv_bfloat16*>(k);
+    nq.heads = static_cast<uint32_t>(B * Hkv);
+    nq.codes = w + L.kc;
+    nq.scales = w + L.ks;
+    nq.vec_ok = aligned(k, 16) ? 1 : 0;
+    if (launch_quantize_rows_nvfp4(nq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    NvColQuantParams vq{};
+    vq.x = static_cast<const __nv_bfloat16*>(v);
+    vq.heads = static_cast<uint32_t>(B * Hkv);
+    vq.rows = static_cast<uint32_t>(N);
+    vq.cols = static_cast<uint32_t>(d);
+    vq.rows_pad = static_cast<uint32_t>(L.npad);
+    vq.codes = w + L.vc;
+    vq.scales = w + L.vs;
+    if (launch_quantize_cols_nvfp4(vq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+    return MXATTN_OK;
   }
   RowQuantParams rq{};
   rq.x = static_cast<const __nv_bfloat16*>(q);
@@ -192,7 +224,8 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
 mxattn_status check_forward_args(const void* q, const void* k, const void* v, const void* out, int B, int Hq,
                                  int Hkv, int N, int d, int scale_mode, int out_dtype, const void* ws,
                                  size_t ws_bytes, WsLayout* L) {
-  if (scale_mode != MXATTN_SCALE_OCP && scale_mode != MXATTN_SCALE_UOS) return MXATTN_ERR_INVALID_ARG;
+  if (scale_mode != MXATTN_SCALE_OCP && scale_mode != MXATTN_SCALE_UOS && scale_mode != MXATTN_SCALE_NVFP4)
+    return MXATTN_ERR_INVALID_ARG;
   if (out_dtype != MXATTN_OUT_F32 && out_dtype != MXATTN_OUT_BF16) return MXATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return MXATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
@@ -429,6 +462,7 @@ mxattn_status mxattn_forward_quantized(const uint8_t* qc, const uint8_t* qs, con
   mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, out, B, Hq, Hkv, N, d, p_scale_mode, out_dtype,
                                        workspace, workspace_bytes, &L);
   if (s != MXATTN_OK) return s;
+  if (p_scale_mode == MXATTN_SCALE_NVFP4) return MXATTN_ERR_UNSUPPORTED;   // MXFP4 operands only
   if (static_cast<uint64_t>(B) * Hq * N >= (1ull << 31)) return MXATTN_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(workspace);

@@ -13,6 +13,10 @@ constexpr int kKvTile = 64;
 
 enum SfLayout : int { kSfRowMajor = 0, kSfAtom = 1 };
 
+// Scale modes (MXATTN_SCALE_* in mxattn.h): MXFP4 with the OCP or the UOS exponent rule, or the
+// NVFP4 comparison format.
+enum : int { kModeOcp = 0, kModeUos = 1, kModeNvfp4 = 2 };
+
 // Blocks of 32 along the contiguous axis of `heads` matrices of [rows, cols] bf16. Rows in
 // [rows, rows_pad) are written as all-zero blocks (codes 0, scale byte 0).
 struct RowQuantParams {
@@ -42,14 +46,29 @@ cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
 
 // NVFP4 (blocks of 16, E4M3 scales) along the contiguous axis: codes [heads*rows][ceil(cols/16)*8],
 // scales [heads*rows][ceil(cols/16)].
+// With sf_layout = kSfAtom: rows [rows, rows_pad) are zero (codes 0, scale 0) and the scales go to
+// atoms [heads][rows_pad/128][ceil(cols/64)][512] (an atom: 128 rows x 4 blocks of 16).
 struct NvQuantParams {
   const __nv_bfloat16* x;
   uint32_t heads, rows, cols;
   uint8_t* codes;
   uint8_t* scales;
   int vec_ok;                                  // cols % 8 == 0 and x 16-byte aligned
+  uint32_t rows_pad;                           // >= rows (codes are [heads][rows_pad][nb * 8])
+  int sf_layout;
 };
 cudaError_t launch_quantize_rows_nvfp4(const NvQuantParams& p, cudaStream_t stream);
+
+// NVFP4 along the row axis of `heads` matrices [rows, cols] (V along keys), written transposed:
+// codes [heads][cols][nblk * 8] with nblk = rows_pad / 16 blocks of 16 rows (blocks past `rows` are
+// zero), scales as atoms [heads][rows_pad / 64][512] (MN index = column < 128, K index = block % 4).
+struct NvColQuantParams {
+  const __nv_bfloat16* x;
+  uint32_t heads, rows, cols, rows_pad;
+  uint8_t* codes;
+  uint8_t* scales;
+};
+cudaError_t launch_quantize_cols_nvfp4(const NvColQuantParams& p, cudaStream_t stream);
 
 // Row-major scale bytes -> 512-byte MMA atoms [heads][tiles][512], zero where the source has no
 // element. transposed = 0: src [heads][rows][kb], atom t holds rows 128t.. and blocks 0..3;

@@ -178,39 +178,98 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(ColQuantParams p) {
 // NVFP4 (comparison format): blocks of 16 along the contiguous axis, scale s = E4M3(amax / 6),
 // elements x / s on the E2M1 grid; both quotients are correctly rounded fp32 divisions, so the
 // grid decisions are taken on the same fp32 values the oracle takes them on. One thread per block.
+// amax -> E4M3 scale byte -> codes of x / s (zero block when the scale rounds to 0)
+__device__ __forceinline__ uint32_t nvfp4_block16(float* v, uint2& codes) {
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
+  const uint32_t byte = e4m3_byte(__fdiv_rn(amax, 6.0f));
+  const float s = e4m3_value(byte);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = (s > 0.f) ? __fdiv_rn(v[k], s) : 0.f;
+  codes = make_uint2(cvt_e2m1x8(v), cvt_e2m1x8(v + 8));
+  return byte;
+}
+
 __global__ void __launch_bounds__(256) quantize_rows_nvfp4_kernel(const NvQuantParams p) {
   const uint32_t nb = (p.cols + 15u) / 16u;
-  const uint64_t total = static_cast<uint64_t>(p.heads) * p.rows * nb;
+  const uint32_t rows_pad = p.rows_pad > p.rows ? p.rows_pad : p.rows;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * rows_pad * nb;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const uint64_t row = i / nb;
-    const uint32_t blk = static_cast<uint32_t>(i - row * nb);
+    const uint64_t prow = i / nb;                       // padded row index over all heads
+    const uint32_t blk = static_cast<uint32_t>(i - prow * nb);
+    const uint64_t head = prow / rows_pad;
+    const uint32_t n = static_cast<uint32_t>(prow - head * rows_pad);
     const uint32_t c0 = blk * 16u;
-    const __nv_bfloat16* src = p.x + row * p.cols + c0;
-    float v[16];
-    if (p.vec_ok && c0 + 16u <= p.cols) {
-      const uint4 r0 = ld_stream_u4(src), r1 = ld_stream_u4(src + 8);
-      bf16x8_to_f32(r0, v);
-      bf16x8_to_f32(r1, v + 8);
-    } else {
+    uint2 codes = make_uint2(0u, 0u);
+    uint32_t byte = 0;
+    if (n < p.rows) {
+      const __nv_bfloat16* src = p.x + (head * p.rows + n) * p.cols + c0;
+      float v[16];
+      if (p.vec_ok && c0 + 16u <= p.cols) {
+        const uint4 r0 = ld_stream_u4(src), r1 = ld_stream_u4(src + 8);
+        bf16x8_to_f32(r0, v);
+        bf16x8_to_f32(r1, v + 8);
+      } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = (c0 + k < p.cols) ? __bfloat162float(src[k]) : 0.f;
+        for (int k = 0; k < 16; ++k) v[k] = (c0 + k < p.cols) ? __bfloat162float(src[k]) : 0.f;
+      }
+      byte = nvfp4_block16(v, codes);
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
-    const uint32_t byte = e4m3_byte(__fdiv_rn(amax, 6.0f));
-    const float s = e4m3_value(byte);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] = (s > 0.f) ? __fdiv_rn(v[k], s) : 0.f;
-    const uint2 codes = make_uint2(cvt_e2m1x8(v), cvt_e2m1x8(v + 8));
-    *reinterpret_cast<uint2*>(p.codes + row * (nb * 8u) + blk * 8u) = codes;
-    p.scales[row * nb + blk] = static_cast<uint8_t>(byte);
+    *reinterpret_cast<uint2*>(p.codes + prow * (nb * 8u) + blk * 8u) = codes;
+    if (p.sf_layout == kSfRowMajor) {
+      p.scales[prow * nb + blk] = static_cast<uint8_t>(byte);
+    } else {
+      const uint32_t ksteps = (nb + 3u) / 4u;
+      const uint64_t atom = (head * (rows_pad / 128u) + (n >> 7)) * ksteps + (blk >> 2);
+      p.scales[atom * 512u + atom_offset(n & 127u, blk & 3u)] = static_cast<uint8_t>(byte);
+    }
   }
 }
 
+// One thread per (head, 16-row block, column), columns fastest: the warp's strided loads of one
+// row segment are contiguous across lanes.
+__global__ void __launch_bounds__(256) quantize_cols_nvfp4_kernel(const NvColQuantParams p) {
+  const uint32_t nblk = p.rows_pad / 16u;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * nblk * p.cols;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t col = static_cast<uint32_t>(i % p.cols);
+    const uint64_t hb = i / p.cols;
+    const uint32_t blk = static_cast<uint32_t>(hb % nblk);
+    const uint64_t head = hb / nblk;
+    const uint32_t r0 = blk * 16u;
+    uint2 codes = make_uint2(0u, 0u);
+    uint32_t byte = 0;
+    if (r0 < p.rows) {
+      float v[16];
+      const __nv_bfloat16* src = p.x + (head * p.rows + r0) * p.cols + col;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = (r0 + k < p.rows) ? __bfloat162float(src[static_cast<size_t>(k) * p.cols]) : 0.f;
+      byte = nvfp4_block16(v, codes);
+    }
+    *reinterpret_cast<uint2*>(p.codes + (head * p.cols + col) * (nblk * 8u) + blk * 8u) = codes;
+    const uint64_t atom = head * (p.rows_pad / 64u) + (blk >> 2);
+    p.scales[atom * 512u + atom_offset(col & 127u, blk & 3u)] = static_cast<uint8_t>(byte);
+  }
+}
+
+cudaError_t launch_quantize_cols_nvfp4(const NvColQuantParams& p, cudaStream_t stream) {
+  const uint64_t total = static_cast<uint64_t>(p.heads) * (p.rows_pad / 16u) * p.cols;
+  if (total == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t want = (total + 255) / 256;
+  const uint64_t cap = static_cast<uint64_t>(sms) * 16;
+  quantize_cols_nvfp4_kernel<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_rows_nvfp4(const NvQuantParams& p, cudaStream_t stream) {
-  const uint64_t total = static_cast<uint64_t>(p.heads) * p.rows * ((p.cols + 15u) / 16u);
+  const uint32_t rows_pad = p.rows_pad > p.rows ? p.rows_pad : p.rows;
+  const uint64_t total = static_cast<uint64_t>(p.heads) * rows_pad * ((p.cols + 15u) / 16u);
   if (total == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

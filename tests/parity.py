@@ -86,8 +86,9 @@ def ws_offsets(B, Hq, Hkv, N, d):
     t = npad // 128
     off = 1024
     names = ["qc", "qs", "kc", "ks", "vc", "vs"]
-    sizes = [B * Hq * npad * d // 2, B * Hq * t * 512, B * Hkv * npad * d // 2, B * Hkv * t * 512,
-             B * Hkv * d * npad // 2, B * Hkv * t * 512]
+    qk_atoms = d // 64 if d >= 128 else 1
+    sizes = [B * Hq * npad * d // 2, B * Hq * t * qk_atoms * 512, B * Hkv * npad * d // 2,
+             B * Hkv * t * qk_atoms * 512, B * Hkv * d * npad // 2, B * Hkv * t * 1024]
     res = {}
     for n, s in zip(names, sizes):
         res[n] = (off, s)

@@ -59,8 +59,9 @@ def _ws_mirror(B, Hq, Hkv, N, d):
     npad = up(N, 128)
     t = npad // 128
     off = 1024
-    for nbytes in (B * Hq * npad * d // 2, B * Hq * t * 512, B * Hkv * npad * d // 2, B * Hkv * t * 512,
-                   B * Hkv * d * npad // 2, B * Hkv * t * 512):
+    qk_atoms = d // 64 if d >= 128 else 1
+    for nbytes in (B * Hq * npad * d // 2, B * Hq * t * qk_atoms * 512, B * Hkv * npad * d // 2,
+                   B * Hkv * t * qk_atoms * 512, B * Hkv * d * npad // 2, B * Hkv * t * 1024):
         off = up(off + nbytes, 1024)
     return off
 
@@ -92,7 +93,7 @@ def test_forward_argument_checks(lib):
     assert call(d=96) == UNSUPPORTED
     assert call(Hq=3) == INVALID
     assert call(N=0) == INVALID
-    assert call(mode=2) == INVALID
+    assert call(mode=3) == INVALID
     assert call(od=5) == INVALID
     assert call(q=None) == INVALID
     assert call(q=FAKE + 2) == INVALID

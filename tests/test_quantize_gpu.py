@@ -100,12 +100,13 @@ def test_forward_prepare_layouts(dev, d, mode):
     for name, t, H in (("q", q, Hq), ("k", k, Hkv)):
         oc, os_ = mx.quantize_rows(pad_rows(t.double().numpy()), mode)
         assert np.array_equal(region(name + "c").reshape(B * H, npad, d // 2), oc.reshape(B * H, npad, d // 2))
-        sf = parity.atom_to_rowmajor(region(name + "s"), B * H, npad, d // 32)
+        # MXFP4 packs one atom per 128 rows at the front of a region sized for NVFP4
+        sf = parity.atom_to_rowmajor(region(name + "s")[:B * H * (npad // 128) * 512], B * H, npad, d // 32)
         assert np.array_equal(sf, os_.reshape(B * H, npad, d // 32))
     oc, os_ = mx.quantize_transposed(pad_rows(v.double().numpy()), mode)      # [B,Hkv,d,npad/2]
     assert np.array_equal(region("vc").reshape(B * Hkv, d, npad // 2), oc.reshape(B * Hkv, d, npad // 2))
     # V scale atoms: MN index = channel, K index = key block inside each 128-key tile
-    a = region("vs").reshape(B * Hkv, npad // 128, 512)
+    a = region("vs")[:B * Hkv * (npad // 128) * 512].reshape(B * Hkv, npad // 128, 512)
     ch = np.arange(d)
     for kb in range(npad // 32):
         got = a[:, kb // 4, (ch % 32) * 16 + (ch // 32) * 4 + kb % 4]
