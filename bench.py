@@ -287,6 +287,21 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     fq_ms = f_start.elapsed_time(f_stop) / fq_steps
     del fq_ops
 
+    # the NVFP4 comparison mode of the same kernel on the same workload (attention kernel alone)
+    api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_NVFP4, ws)
+    for _ in range(2):
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_NVFP4, True, ws)
+    barrier()
+    n_start, n_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_start.record(stream)
+    for _ in range(fq_steps):
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_NVFP4, True, ws)
+    n_stop.record(stream)
+    barrier()
+    if api.mxattn_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout in the NVFP4 attention")
+    nv_attn_ms = n_start.elapsed_time(n_stop) / fq_steps
+
     # block-scaled MXFP4 GEMM (W4A4) on its own workload: A [M, K], B [N, K] quantized once
     gm, gn, gk = synthetic.GEMM_SHAPE
     ga = torch.randn((gm, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(5))
@@ -339,8 +354,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
-    step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms = reduce_max_over_ranks(
-        [total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms], world, dev)
+    (step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
+     nv_attn_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms,
+                                          gemm_ms, gemm_nv_ms, nv_attn_ms], world, dev)
     if rank != 0:
         return
 
@@ -379,6 +395,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                       "standalone_ms": quant_alone_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
                       "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
+        "nvfp4_attention": {"ms": nv_attn_ms, "tflops": flops / (nv_attn_ms * 1e-3) / 1e12,
+                            "note": "MXATTN_SCALE_NVFP4 (Q, K, V, P~ in NVFP4), attention kernel alone"},
         "forward_quantized": {"ms": fq_ms, "tflops": flops / (fq_ms * 1e-3) / 1e12,
                               "note": "mxattn_forward_quantized on pre-quantized Q/K/V: scale repack + kernel"},
         "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
