@@ -29,7 +29,10 @@
 //              quantizes it in registers, writes codes (32B-swizzled, the MMA operand layout)
 //              and scale bytes to shared memory, rescales O and L in TMEM when the max moves,
 //              and finally normalises and stores the output.
-// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..235.
+// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..243.
+// The kernel is templated on the format: MXFP4 (the method) or, for comparison, NVFP4 (blocks of
+// 16 with E4M3 scales for Q, K, V and P~; kind::mxf4nvf4 products, the non-power-of-two P~ scale
+// folded into the exponent bias as -log2 s).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>

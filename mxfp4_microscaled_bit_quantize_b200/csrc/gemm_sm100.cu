@@ -10,7 +10,7 @@
 // Persistent kernel: one CTA per SM walks 128 x 256 tiles of C in groups of kGroupM tile rows
 // (so the A and B slices in flight at once stay in L2). Roles:
 //   warp 0     TMA producer: K slices of 256 elements (128 bytes of codes per row) of A (128 rows)
-//              and B (256 rows), 128-byte swizzle, into a kGStages-deep ring that runs across
+//              and B (256 rows), 128-byte swizzle, into a 4-stage (NVFP4: 3) ring that runs across
 //              tile boundaries, plus their scale atoms (512 bytes per 128 rows x 128 K elements).
 //   warp 1     TMEM owner and MMA issuer: tcgen05.cp moves the scale atoms of a stage into that
 //              stage's own TMEM columns (a copy is not ordered behind earlier MMAs that read the
@@ -22,7 +22,9 @@
 //              registers (packed bf16), release the accumulator, then stream the row out through a
 //              128-byte-swizzled staging box in shared memory, one TMA store per 64 columns, while
 //              the next tile's MMAs run. fp32: direct row stores, then release.
-// TMEM: accumulator columns [0, 256), scale columns from 256 (kGStages x 24).
+// TMEM: accumulator columns [0, 256), scale columns from 256 (12 per scale atom of a stage).
+// Templated on the format: MXFP4 (blocks of 32, UE8M0, kind::mxf4) or NVFP4 (blocks of 16, UE4M3,
+// kind::mxf4nvf4: twice the scale atoms per K, so a 3-stage ring).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>

@@ -288,16 +288,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // Two fp32 values -> one byte of E2M1 codes (round to nearest even, saturating at 6);
 // `lo` lands in bits 0..3, `hi` in bits 4..7.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(hi), "f"(lo));
-  return out & 0xFFu;
-}
-
 // Non-negative fp32 -> unsigned FP8 E4M3 byte, round to nearest-even, saturating at 448 (the
 // hardware conversion; the first source operand lands in the upper byte of the pair).
 __device__ __forceinline__ uint32_t e4m3_byte(float v) {
