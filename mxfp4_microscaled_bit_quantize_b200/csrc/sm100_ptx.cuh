@@ -286,8 +286,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // ------------------------------------------------------------------ E2M1 conversion
 
-// Two fp32 values -> one byte of E2M1 codes (round to nearest even, saturating at 6);
-// `lo` lands in bits 0..3, `hi` in bits 4..7.
 // Non-negative fp32 -> unsigned FP8 E4M3 byte, round to nearest-even, saturating at 448 (the
 // hardware conversion; the first source operand lands in the upper byte of the pair).
 __device__ __forceinline__ uint32_t e4m3_byte(float v) {
