@@ -179,6 +179,23 @@ mxattn_status mxattn_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mxattn_forward_host -- mxattn_forward on HOST buffers (same arguments; q, k, v, out are host
+ * pointers, best page-locked so the copies run asynchronously). The work is split into groups of
+ * consecutive KV heads (with their query heads) that flow through two device slots: a group's
+ * inputs are copied in on a library-owned stream while the previous group is quantized and
+ * attended on `stream` and the one before is copied out on a second library-owned stream, so the
+ * host<->device transfers overlap the kernels. Heads are independent: the output is bit-identical
+ * to mxattn_forward's. The call is asynchronous on `stream`: the output is in `out` once `stream`
+ * has reached this point. Device workspace: mxattn_forward_host_workspace_size(..., out_dtype)
+ * bytes, 256-byte aligned; its first word is the status word read by mxattn_check_status.
+ * Errors: as mxattn_forward (MXATTN_ERR_WORKSPACE against the host workspace size).
+ */
+size_t mxattn_forward_host_workspace_size(int B, int Hq, int Hkv, int N, int d, int out_dtype);
+mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                                  int N, int d, int causal, int scale_mode, int pnq, int out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * The two halves of mxattn_forward, for callers that time or reuse them separately:
  *   mxattn_forward_prepare quantizes q, k, v into the workspace;
  *   mxattn_forward_attend runs the fused attention kernel on a prepared workspace (same

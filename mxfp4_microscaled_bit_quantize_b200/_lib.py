@@ -24,6 +24,8 @@ SIGNATURES = {
     "mxattn_forward_debug": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 9 + [_vp, _c_size, _vp]
                              + [_c_int] * 3 + [_u8p, _u8p]),
     "mxattn_forward_noalloc": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 9 + [_vp]),
+    "mxattn_forward_host_workspace_size": (_c_size, [_c_int] * 6),
+    "mxattn_forward_host": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 9 + [_vp, _c_size, _vp]),
     "mxattn_forward_quantized": (_c_int, [_u8p] * 6 + [_vp] + [_c_int] * 9 + [_vp, _c_size, _vp]),
     "mxattn_gemm_workspace_size": (_c_size, [_c_i64] * 3),
     "mxattn_gemm": (_c_int, [_u8p] * 4 + [_vp] + [_c_i64] * 3 + [_c_int, _vp, _c_size, _vp]),

@@ -107,6 +107,35 @@ def mxattn_forward(q, k, v, causal: bool = False, scale_mode: int = SCALE_UOS, p
     return out
 
 
+def mxattn_forward_host(q, k, v, out, causal: bool = False, scale_mode: int = SCALE_UOS, pnq: bool = True,
+                        workspace: torch.Tensor | None = None, device=None) -> torch.Tensor:
+    """mxattn_forward on host (CPU, ideally pinned) bf16 tensors q [B,Hq,N,d], k/v [B,Hkv,N,d] and a host
+    output tensor out [B,Hq,N,d] (fp32 or bf16): copies and kernels are pipelined over groups of
+    KV heads. Asynchronous on the device's current stream; synchronise before reading `out`."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous bf16 host tensor")
+    if out.is_cuda or not out.is_contiguous() or out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out must be a contiguous fp32 or bf16 host tensor")
+    B, Hq, N, d = (int(x) for x in q.shape)
+    Hkv = int(k.shape[1])
+    if tuple(k.shape) != tuple(v.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shapes must be q/out [B,Hq,N,d], k/v [B,Hkv,N,d]")
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    lib = _lib.load()
+    if workspace is None:
+        n = int(lib.mxattn_forward_host_workspace_size(B, Hq, Hkv, N, d, od))
+        if n == 0:
+            raise ValueError("unsupported attention shape")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    st = lib.mxattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                                 int(bool(causal)), int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                                 workspace.numel(), _stream(dev))
+    _lib.check(st, "mxattn_forward_host")
+    return out
+
+
 def mxattn_forward_quantized(qc, qs, kc, ks, vtc, vts, N: int, d: int, causal: bool = False,
                              p_scale_mode: int = SCALE_UOS, pnq: bool = True, out_dtype=torch.float32,
                              workspace: torch.Tensor | None = None, out: torch.Tensor | None = None):

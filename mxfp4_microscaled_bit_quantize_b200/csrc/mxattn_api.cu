@@ -7,6 +7,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "../../include/mxattn.h"
 #include "mxattn_internal.h"
@@ -98,7 +100,6 @@ bool make_map_typed(CUtensorMap* m, CUtensorMapDataType dtype, const void* base,
 mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                            int scale_mode, void* ws, size_t ws_bytes, cudaStream_t st, const WsLayout& L) {
   uint8_t* w = static_cast<uint8_t*>(ws);
-  if (cudaMemsetAsync(w, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
   if (d < kTile) {
     // scale atoms have room for 128 rows / 4 blocks; d = 64 leaves part of them unused
     if (cudaMemsetAsync(w + L.qs, 0, L.kc - L.qs, st) != cudaSuccess) return MXATTN_ERR_CUDA;
@@ -186,7 +187,8 @@ CodeSources workspace_codes(void* ws, const WsLayout& L) {
 
 mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int causal, int scale_mode, int pnq,
                           int out_dtype, void* ws, cudaStream_t st, const WsLayout& L, const CodeSources& src,
-                          int dbg_bh, int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales) {
+                          int dbg_bh, int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales,
+                          unsigned int* status = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -212,7 +214,7 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   p.mode = scale_mode;
   p.pnq = pnq ? 1 : 0;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
-  p.status = reinterpret_cast<unsigned int*>(w);
+  p.status = status ? status : reinterpret_cast<unsigned int*>(w);
   p.dbg_codes = p_codes;
   p.dbg_scales = p_scales;
   p.dbg_bh = dbg_bh;
@@ -435,6 +437,7 @@ mxattn_status mxattn_forward_prepare(const void* q, const void* k, const void* v
   mxattn_status s = check_forward_args(q, k, v, nullptr, B, Hq, Hkv, N, d, scale_mode, MXATTN_OUT_F32, workspace,
                                        workspace_bytes, &L);
   if (s != MXATTN_OK) return s;
+  if (cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MXATTN_ERR_CUDA;
   return prepare_impl(q, k, v, B, Hq, Hkv, N, d, scale_mode, workspace, workspace_bytes,
                       static_cast<cudaStream_t>(stream), L);
 }
@@ -502,10 +505,151 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
       return MXATTN_ERR_INVALID_ARG;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 256, st) != cudaSuccess) return MXATTN_ERR_CUDA;
   s = prepare_impl(q, k, v, B, Hq, Hkv, N, d, scale_mode, workspace, workspace_bytes, st, L);
   if (s != MXATTN_OK) return s;
   return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace, st, L,
                      workspace_codes(workspace, L), dbg_bh, dbg_r0, dbg_r1, p_codes, p_scales);
+}
+
+// ---------------------------------------------------------------- host-buffer pipeline
+// mxattn_forward on host buffers: KV-head groups ("chunks") flow through two device slots. Per
+// chunk, the inputs are copied in on one stream, quantized and attended on the caller's stream,
+// and the output copied out on a third, so copies in both directions overlap the kernels of
+// neighbouring chunks. Heads are independent, so the result equals mxattn_forward's.
+
+struct HostPlan {
+  int cg;                  // KV heads per chunk (the slots are sized for it)
+  std::vector<int> sizes;  // KV heads per chunk, in order
+  size_t q_bytes, kv_bytes, out_bytes, attn_ws;   // per slot, for a full chunk
+  size_t slot_bytes, total;
+};
+
+static bool host_plan(int B, int Hq, int Hkv, int N, int d, int out_dtype, HostPlan* P) {
+  WsLayout L;
+  if (!ws_layout(B, Hq, Hkv, N, d, &L)) return false;
+  if (out_dtype != MXATTN_OUT_F32 && out_dtype != MXATTN_OUT_BF16) return false;
+  const int group = Hq / Hkv;
+  const int units = B * Hkv;
+  const long n_qt = (N + kTile - 1) / kTile;
+  const long target_ctas = 2048;   // about seven waves of two CTAs per SM: small tail per chunk
+  long cg = (target_ctas + group * n_qt - 1) / (group * n_qt);
+  if (cg < 1) cg = 1;
+  if (cg > units) cg = units;
+  P->cg = static_cast<int>(cg);
+  // equal chunks (the last may be smaller): measured on the video-DiT shape, the copies bound the
+  // pipeline, and a schedule that ramps the chunk size up and down was no faster
+  P->sizes.clear();
+  for (int u = 0; u < units; u += static_cast<int>(cg))
+    P->sizes.push_back(u + cg <= units ? static_cast<int>(cg) : units - u);
+  const size_t hd = static_cast<size_t>(N) * d;
+  P->q_bytes = static_cast<size_t>(cg) * group * hd * 2;
+  P->kv_bytes = static_cast<size_t>(cg) * hd * 2;
+  P->out_bytes = static_cast<size_t>(cg) * group * hd * (out_dtype == MXATTN_OUT_F32 ? 4 : 2);
+  WsLayout Lc;
+  if (!ws_layout(1, static_cast<int>(cg) * group, static_cast<int>(cg), N, d, &Lc)) return false;
+  P->attn_ws = Lc.total;
+  P->slot_bytes = align_up(P->q_bytes, kAlign) + 2 * align_up(P->kv_bytes, kAlign) + align_up(P->out_bytes, kAlign) +
+                  align_up(P->attn_ws, kAlign);
+  P->total = kAlign + 2 * P->slot_bytes;
+  return true;
+}
+
+struct SideStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+};
+
+static mxattn_status side_streams(SideStreams* out) {
+  static std::mutex mu;
+  static SideStreams cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MXATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  SideStreams& c = cache[dev];
+  if (!c.in && cudaStreamCreateWithFlags(&c.in, cudaStreamNonBlocking) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (!c.out && cudaStreamCreateWithFlags(&c.out, cudaStreamNonBlocking) != cudaSuccess) return MXATTN_ERR_CUDA;
+  *out = c;
+  return MXATTN_OK;
+}
+
+size_t mxattn_forward_host_workspace_size(int B, int Hq, int Hkv, int N, int d, int out_dtype) {
+  HostPlan P;
+  return host_plan(B, Hq, Hkv, N, d, out_dtype, &P) ? P.total : 0;
+}
+
+mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                                  int N, int d, int causal, int scale_mode, int pnq, int out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out) return MXATTN_ERR_INVALID_ARG;
+  WsLayout L;
+  mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, N, d, scale_mode, out_dtype,
+                                       workspace, workspace_bytes, &L);
+  if (s != MXATTN_OK && s != MXATTN_ERR_WORKSPACE) return s;
+  HostPlan P;
+  if (!host_plan(B, Hq, Hkv, N, d, out_dtype, &P)) return MXATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < P.total) return MXATTN_ERR_WORKSPACE;
+  SideStreams ss;
+  if ((s = side_streams(&ss)) != MXATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  unsigned int* status = reinterpret_cast<unsigned int*>(w);
+  const int group = Hq / Hkv;
+  const size_t hd = static_cast<size_t>(N) * d;
+  const size_t out_elem = (out_dtype == MXATTN_OUT_F32) ? 4 : 2;
+
+  // events: start (orders the side streams after earlier work on the caller's stream), and per
+  // chunk inputs-in, compute-done, output-out
+  const int chunks = static_cast<int>(P.sizes.size());
+  std::vector<cudaEvent_t> ev(1 + 3 * static_cast<size_t>(chunks), nullptr);
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) s = MXATTN_ERR_CUDA;
+  auto ev_in = [&](int c) { return ev[1 + 3 * c]; };
+  auto ev_comp = [&](int c) { return ev[2 + 3 * c]; };
+  auto ev_out = [&](int c) { return ev[3 + 3 * c]; };
+  auto ok = [&](cudaError_t e) { if (e != cudaSuccess && s == MXATTN_OK) s = MXATTN_ERR_CUDA; };
+  if (s == MXATTN_OK) {
+    ok(cudaMemsetAsync(w, 0, 256, st));
+    ok(cudaEventRecord(ev[0], st));
+    ok(cudaStreamWaitEvent(ss.in, ev[0], 0));
+    ok(cudaStreamWaitEvent(ss.out, ev[0], 0));
+  }
+  int u0 = 0;
+  for (int c = 0; c < chunks && s == MXATTN_OK; u0 += P.sizes[c], ++c) {
+    const int cu = P.sizes[c];                                   // KV heads in this chunk
+    uint8_t* slot = w + kAlign + static_cast<size_t>(c & 1) * P.slot_bytes;
+    uint8_t* dq = slot;
+    uint8_t* dk = dq + align_up(P.q_bytes, kAlign);
+    uint8_t* dv = dk + align_up(P.kv_bytes, kAlign);
+    uint8_t* dout = dv + align_up(P.kv_bytes, kAlign);
+    uint8_t* aws = dout + align_up(P.out_bytes, kAlign);
+    const size_t qb = static_cast<size_t>(cu) * group * hd * 2, kvb = static_cast<size_t>(cu) * hd * 2;
+    const size_t ob = static_cast<size_t>(cu) * group * hd * out_elem;
+    const size_t q_off = static_cast<size_t>(u0) * group * hd, kv_off = static_cast<size_t>(u0) * hd;
+    // inputs: the slot is free once the output of chunk c-2 has left it
+    if (c >= 2) ok(cudaStreamWaitEvent(ss.in, ev_out(c - 2), 0));
+    ok(cudaMemcpyAsync(dq, static_cast<const uint8_t*>(q) + q_off * 2, qb, cudaMemcpyHostToDevice, ss.in));
+    ok(cudaMemcpyAsync(dk, static_cast<const uint8_t*>(k) + kv_off * 2, kvb, cudaMemcpyHostToDevice, ss.in));
+    ok(cudaMemcpyAsync(dv, static_cast<const uint8_t*>(v) + kv_off * 2, kvb, cudaMemcpyHostToDevice, ss.in));
+    ok(cudaEventRecord(ev_in(c), ss.in));
+    // compute on the caller's stream
+    ok(cudaStreamWaitEvent(st, ev_in(c), 0));
+    WsLayout Lc;
+    ws_layout(1, cu * group, cu, N, d, &Lc);
+    if (s == MXATTN_OK) s = prepare_impl(dq, dk, dv, 1, cu * group, cu, N, d, scale_mode, aws, P.attn_ws, st, Lc);
+    if (s == MXATTN_OK)
+      s = attend_impl(dout, 1, cu * group, cu, N, d, causal, scale_mode, pnq, out_dtype, aws, st, Lc,
+                      workspace_codes(aws, Lc), -1, 0, 0, nullptr, nullptr, status);
+    ok(cudaEventRecord(ev_comp(c), st));
+    // output
+    ok(cudaStreamWaitEvent(ss.out, ev_comp(c), 0));
+    ok(cudaMemcpyAsync(static_cast<uint8_t*>(out) + q_off * out_elem, dout, ob, cudaMemcpyDeviceToHost, ss.out));
+    ok(cudaEventRecord(ev_out(c), ss.out));
+  }
+  // the call completes on the caller's stream once the last output has been copied out
+  if (s == MXATTN_OK) ok(cudaStreamWaitEvent(st, ev_out(chunks - 1), 0));
+  for (auto& e : ev)
+    if (e) cudaEventDestroy(e);   // released once recorded work completes
+  return s;
 }
 
 mxattn_status mxattn_selftest_wait_timeout(void* workspace, void* stream) {
