@@ -421,6 +421,15 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                                 "kind": "oracle",
                                 "sample": f"{args.cpu_rows} query rows of head 0 (that head's Q/K/V "
                                           f"quantized, attention over all {cfg.N} keys), {dt:.1f} s"}
+        try:   # the same oracle on one thread (BLAS limited to 1), on an eighth of the rows
+            from threadpoolctl import threadpool_limits
+            rows1 = max(64, args.cpu_rows // 8)
+            with threadpool_limits(limits=1):
+                f1, dt1 = oracle_sample(cfg, rows1)
+            line["cpu_baseline"]["single_thread"] = {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s", "rows": rows1,
+                                                     "seconds": dt1}
+        except ImportError:
+            pass
     print(json.dumps(line), flush=True)
 
 
