@@ -270,6 +270,36 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     e2e_ms = e_start.elapsed_time(e_stop) / e2e_steps
     del host_ws
 
+    # the floor for any pipeline over this host link: the same bytes copied both ways at once
+    # (inputs in, output out, on two streams), with no kernels
+    link_in, link_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    staging = torch.empty(h2d, dtype=torch.uint8, device=dev)
+
+    def both_ways():
+        link_in.wait_stream(stream)
+        link_out.wait_stream(stream)
+        with torch.cuda.stream(link_in):
+            o = 0
+            for t in (q_h, k_h, v_h):
+                nb = t.numel() * t.element_size()
+                staging[o:o + nb].copy_(t.view(-1).view(torch.uint8), non_blocking=True)
+                o += nb
+        with torch.cuda.stream(link_out):
+            out_h.copy_(out, non_blocking=True)
+        stream.wait_stream(link_in)
+        stream.wait_stream(link_out)
+
+    both_ways()
+    barrier()
+    c_start, c_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c_start.record(stream)
+    for _ in range(3):
+        both_ways()
+    c_stop.record(stream)
+    barrier()
+    copy_ms = c_start.elapsed_time(c_stop) / 3
+    del staging
+
     # the attention kernel on caller-owned MXFP4 operands (mxattn_forward_quantized): scale
     # repacking + the fused kernel, with the codes quantized once outside the timed loop
     fq_ops = (*api.mxattn_quantize(dq, False, api.SCALE_UOS), *api.mxattn_quantize(dk, False, api.SCALE_UOS),
@@ -356,9 +386,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
-    (step_ms, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
-     nv_attn_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, quant_alone_ms, fq_ms,
-                                          gemm_ms, gemm_nv_ms, nv_attn_ms], world, dev)
+    (step_ms, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
+     nv_attn_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms,
+                                          fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms], world, dev)
     if rank != 0:
         return
 
@@ -411,7 +441,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                                                                    sources_hash(GEMM_SOURCES))}},
         "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "api": "mxattn_forward_host (pinned host buffers in and out)"},
+                "api": "mxattn_forward_host (pinned host buffers in and out)",
+                "copy_floor": {"ms": copy_ms, "gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
+                               "frac": copy_ms / e2e_ms,
+                               "note": "the same H2D and D2H bytes copied concurrently, no kernels"}},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks.summary(),
     }

@@ -181,13 +181,18 @@ mxattn_status mxattn_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
 /*
  * mxattn_forward_host -- mxattn_forward on HOST buffers (same arguments; q, k, v, out are host
  * pointers, best page-locked so the copies run asynchronously). The work is split into groups of
- * consecutive KV heads (with their query heads) that flow through two device slots: a group's
- * inputs are copied in on a library-owned stream while the previous group is quantized and
- * attended on `stream` and the one before is copied out on a second library-owned stream, so the
- * host<->device transfers overlap the kernels. Heads are independent: the output is bit-identical
- * to mxattn_forward's. The call is asynchronous on `stream`: the output is in `out` once `stream`
- * has reached this point. Device workspace: mxattn_forward_host_workspace_size(..., out_dtype)
- * bytes, 256-byte aligned; its first word is the status word read by mxattn_check_status.
+ * consecutive KV heads (with their query heads, about 512 attention CTAs per group) that rotate
+ * through three device slots. Inputs are copied in on a library-owned stream; each group is
+ * quantized and attended on `stream` or on a library-owned second compute stream, alternately;
+ * outputs are copied out on a third library-owned stream. A slot's input buffers are refilled as
+ * soon as its quantizers have read them, so copies run in both directions at once and overlap
+ * the kernels. Heads are independent: the output is bit-identical to mxattn_forward's. The call
+ * is asynchronous on `stream`: it starts after the work already queued there, and the output is
+ * in `out` once `stream` has reached this point. Concurrent calls on one device (each with its
+ * own workspace) share the library's streams: their copies and kernels interleave on them, and
+ * each stays correct, since every wait is on an event recorded before it. Device workspace:
+ * mxattn_forward_host_workspace_size(..., out_dtype) bytes, 256-byte aligned; its first word is
+ * the status word read by mxattn_check_status.
  * Errors: as mxattn_forward (MXATTN_ERR_WORKSPACE against the host workspace size).
  */
 size_t mxattn_forward_host_workspace_size(int B, int Hq, int Hkv, int N, int d, int out_dtype);

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -513,10 +514,17 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
 }
 
 // ---------------------------------------------------------------- host-buffer pipeline
-// mxattn_forward on host buffers: KV-head groups ("chunks") flow through two device slots. Per
-// chunk, the inputs are copied in on one stream, quantized and attended on the caller's stream,
-// and the output copied out on a third, so copies in both directions overlap the kernels of
-// neighbouring chunks. Heads are independent, so the result equals mxattn_forward's.
+// mxattn_forward on host buffers: KV-head groups ("chunks") flow through kHostSlots device slots.
+// Per chunk, the inputs are copied in on one stream, quantized and attended on one of two compute
+// streams (the caller's and a side stream, alternating by chunk), and the output is copied out on
+// a fourth. Each part of a slot is reused as soon as its last reader is done: the bf16 inputs once
+// the quantizers have read them, the codes once the attention kernel has, the output once it has
+// been copied out. So the host-to-device stream runs back to back while the device-to-host copies
+// go the other way, and the attention kernel of one chunk fills the SMs that the tail of the
+// previous chunk's kernel leaves idle. Heads are independent, so the result equals mxattn_forward's.
+
+constexpr int kHostSlots = 3;          // device slots the chunks rotate through
+constexpr long kHostChunkCtas = 512;   // attention CTAs per chunk (rounded up to whole KV heads)
 
 struct HostPlan {
   int cg;                  // KV heads per chunk (the slots are sized for it)
@@ -532,16 +540,23 @@ static bool host_plan(int B, int Hq, int Hkv, int N, int d, int out_dtype, HostP
   const int group = Hq / Hkv;
   const int units = B * Hkv;
   const long n_qt = (N + kTile - 1) / kTile;
-  const long target_ctas = 2048;   // about seven waves of two CTAs per SM: small tail per chunk
+  // small chunks keep the pipeline's fill (the first chunk's copy-in) and drain (the last chunk's
+  // kernel and copy-out) short; the wave tail of each chunk's kernel is filled by the next chunk's
+  // kernel on the other compute stream
+  const long target_ctas = kHostChunkCtas;
   long cg = (target_ctas + group * n_qt - 1) / (group * n_qt);
   if (cg < 1) cg = 1;
   if (cg > units) cg = units;
   P->cg = static_cast<int>(cg);
-  // equal chunks (the last may be smaller): measured on the video-DiT shape, the copies bound the
-  // pipeline, and a schedule that ramps the chunk size up and down was no faster
+  // full chunks, except that the first and the last hold half a chunk when there are more than
+  // two: a shorter first copy-in and a shorter last kernel and copy-out trim the fill and the
+  // drain (1% on the video-DiT shape)
   P->sizes.clear();
-  for (int u = 0; u < units; u += static_cast<int>(cg))
-    P->sizes.push_back(u + cg <= units ? static_cast<int>(cg) : units - u);
+  const int full = static_cast<int>(cg);
+  const int edge = units > 2 * full ? (full > 1 ? full / 2 : 1) : 0;
+  if (edge) P->sizes.push_back(edge);
+  for (int u = edge; u < units - edge; u += full) P->sizes.push_back(std::min(full, units - edge - u));
+  if (edge) P->sizes.push_back(edge);
   const size_t hd = static_cast<size_t>(N) * d;
   P->q_bytes = static_cast<size_t>(cg) * group * hd * 2;
   P->kv_bytes = static_cast<size_t>(cg) * hd * 2;
@@ -551,12 +566,12 @@ static bool host_plan(int B, int Hq, int Hkv, int N, int d, int out_dtype, HostP
   P->attn_ws = Lc.total;
   P->slot_bytes = align_up(P->q_bytes, kAlign) + 2 * align_up(P->kv_bytes, kAlign) + align_up(P->out_bytes, kAlign) +
                   align_up(P->attn_ws, kAlign);
-  P->total = kAlign + 2 * P->slot_bytes;
+  P->total = kAlign + kHostSlots * P->slot_bytes;
   return true;
 }
 
 struct SideStreams {
-  cudaStream_t in = nullptr, out = nullptr;
+  cudaStream_t in = nullptr, out = nullptr, comp = nullptr;
 };
 
 static mxattn_status side_streams(SideStreams* out) {
@@ -568,6 +583,7 @@ static mxattn_status side_streams(SideStreams* out) {
   SideStreams& c = cache[dev];
   if (!c.in && cudaStreamCreateWithFlags(&c.in, cudaStreamNonBlocking) != cudaSuccess) return MXATTN_ERR_CUDA;
   if (!c.out && cudaStreamCreateWithFlags(&c.out, cudaStreamNonBlocking) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (!c.comp && cudaStreamCreateWithFlags(&c.comp, cudaStreamNonBlocking) != cudaSuccess) return MXATTN_ERR_CUDA;
   *out = c;
   return MXATTN_OK;
 }
@@ -598,25 +614,29 @@ mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, v
   const size_t out_elem = (out_dtype == MXATTN_OUT_F32) ? 4 : 2;
 
   // events: start (orders the side streams after earlier work on the caller's stream), and per
-  // chunk inputs-in, compute-done, output-out
+  // chunk inputs-in, inputs-consumed, compute-done, output-out
   const int chunks = static_cast<int>(P.sizes.size());
-  std::vector<cudaEvent_t> ev(1 + 3 * static_cast<size_t>(chunks), nullptr);
+  std::vector<cudaEvent_t> ev(1 + 4 * static_cast<size_t>(chunks), nullptr);
   for (auto& e : ev)
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) s = MXATTN_ERR_CUDA;
-  auto ev_in = [&](int c) { return ev[1 + 3 * c]; };
-  auto ev_comp = [&](int c) { return ev[2 + 3 * c]; };
-  auto ev_out = [&](int c) { return ev[3 + 3 * c]; };
+  auto ev_in = [&](int c) { return ev[1 + 4 * c]; };
+  auto ev_prep = [&](int c) { return ev[2 + 4 * c]; };
+  auto ev_comp = [&](int c) { return ev[3 + 4 * c]; };
+  auto ev_out = [&](int c) { return ev[4 + 4 * c]; };
   auto ok = [&](cudaError_t e) { if (e != cudaSuccess && s == MXATTN_OK) s = MXATTN_ERR_CUDA; };
   if (s == MXATTN_OK) {
     ok(cudaMemsetAsync(w, 0, 256, st));
     ok(cudaEventRecord(ev[0], st));
     ok(cudaStreamWaitEvent(ss.in, ev[0], 0));
     ok(cudaStreamWaitEvent(ss.out, ev[0], 0));
+    ok(cudaStreamWaitEvent(ss.comp, ev[0], 0));
   }
   int u0 = 0;
   for (int c = 0; c < chunks && s == MXATTN_OK; u0 += P.sizes[c], ++c) {
     const int cu = P.sizes[c];                                   // KV heads in this chunk
-    uint8_t* slot = w + kAlign + static_cast<size_t>(c & 1) * P.slot_bytes;
+    const bool reuse = c >= kHostSlots;                          // the slot held chunk c - kHostSlots
+    cudaStream_t cs = (c & 1) ? ss.comp : st;
+    uint8_t* slot = w + kAlign + static_cast<size_t>(c % kHostSlots) * P.slot_bytes;
     uint8_t* dq = slot;
     uint8_t* dk = dq + align_up(P.q_bytes, kAlign);
     uint8_t* dv = dk + align_up(P.kv_bytes, kAlign);
@@ -625,27 +645,32 @@ mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, v
     const size_t qb = static_cast<size_t>(cu) * group * hd * 2, kvb = static_cast<size_t>(cu) * hd * 2;
     const size_t ob = static_cast<size_t>(cu) * group * hd * out_elem;
     const size_t q_off = static_cast<size_t>(u0) * group * hd, kv_off = static_cast<size_t>(u0) * hd;
-    // inputs: the slot is free once the output of chunk c-2 has left it
-    if (c >= 2) ok(cudaStreamWaitEvent(ss.in, ev_out(c - 2), 0));
+    // inputs, once the quantizers of the slot's previous chunk have read its bf16 buffers
+    if (reuse) ok(cudaStreamWaitEvent(ss.in, ev_prep(c - kHostSlots), 0));
     ok(cudaMemcpyAsync(dq, static_cast<const uint8_t*>(q) + q_off * 2, qb, cudaMemcpyHostToDevice, ss.in));
     ok(cudaMemcpyAsync(dk, static_cast<const uint8_t*>(k) + kv_off * 2, kvb, cudaMemcpyHostToDevice, ss.in));
     ok(cudaMemcpyAsync(dv, static_cast<const uint8_t*>(v) + kv_off * 2, kvb, cudaMemcpyHostToDevice, ss.in));
     ok(cudaEventRecord(ev_in(c), ss.in));
-    // compute on the caller's stream
-    ok(cudaStreamWaitEvent(st, ev_in(c), 0));
+    // quantizers: the codes region is free once the previous chunk's attention kernel has read it
+    ok(cudaStreamWaitEvent(cs, ev_in(c), 0));
+    if (reuse) ok(cudaStreamWaitEvent(cs, ev_comp(c - kHostSlots), 0));
     WsLayout Lc;
     ws_layout(1, cu * group, cu, N, d, &Lc);
-    if (s == MXATTN_OK) s = prepare_impl(dq, dk, dv, 1, cu * group, cu, N, d, scale_mode, aws, P.attn_ws, st, Lc);
+    if (s == MXATTN_OK) s = prepare_impl(dq, dk, dv, 1, cu * group, cu, N, d, scale_mode, aws, P.attn_ws, cs, Lc);
+    ok(cudaEventRecord(ev_prep(c), cs));
+    // attention: the output buffer is free once the previous chunk's output has been copied out
+    if (reuse) ok(cudaStreamWaitEvent(cs, ev_out(c - kHostSlots), 0));
     if (s == MXATTN_OK)
-      s = attend_impl(dout, 1, cu * group, cu, N, d, causal, scale_mode, pnq, out_dtype, aws, st, Lc,
+      s = attend_impl(dout, 1, cu * group, cu, N, d, causal, scale_mode, pnq, out_dtype, aws, cs, Lc,
                       workspace_codes(aws, Lc), -1, 0, 0, nullptr, nullptr, status);
-    ok(cudaEventRecord(ev_comp(c), st));
+    ok(cudaEventRecord(ev_comp(c), cs));
     // output
     ok(cudaStreamWaitEvent(ss.out, ev_comp(c), 0));
     ok(cudaMemcpyAsync(static_cast<uint8_t*>(out) + q_off * out_elem, dout, ob, cudaMemcpyDeviceToHost, ss.out));
     ok(cudaEventRecord(ev_out(c), ss.out));
   }
-  // the call completes on the caller's stream once the last output has been copied out
+  // the call completes on the caller's stream once the last output has been copied out (each
+  // copy-out waited for its chunk's kernels, and the copy-out stream runs in chunk order)
   if (s == MXATTN_OK) ok(cudaStreamWaitEvent(st, ev_out(chunks - 1), 0));
   for (auto& e : ev)
     if (e) cudaEventDestroy(e);   // released once recorded work completes

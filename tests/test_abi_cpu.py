@@ -79,6 +79,48 @@ def test_workspace_size_rejects_bad_shapes(lib):
     assert ws(1, 2, 2, 0, 64) == 0
 
 
+def _host_ws_mirror(B, Hq, Hkv, N, d, out_bytes):
+    """Three device slots, each holding one chunk of KV heads: bf16 Q, K, V, the output and the
+    chunk's own attention workspace. A chunk covers about 512 attention CTAs (whole KV heads)."""
+    up = lambda x, a: -(-x // a) * a  # noqa: E731
+    group, units, n_qt = Hq // Hkv, B * Hkv, -(-N // 128)
+    cg = min(max(-(-512 // (group * n_qt)), 1), units)
+    hd = N * d
+    slot = (up(cg * group * hd * 2, 1024) + 2 * up(cg * hd * 2, 1024) + up(cg * group * hd * out_bytes, 1024)
+            + up(_ws_mirror(1, cg * group, cg, N, d), 1024))
+    return 1024 + 3 * slot
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 256, 64), (1, 40, 40, 32760, 128), (4, 32, 8, 8192, 128),
+                                   (1, 24, 24, 76800, 128), (2, 3, 1, 1, 64)])
+def test_host_workspace_size(lib, shape):
+    hw = lib.mxattn_forward_host_workspace_size
+    assert hw(*shape, 0) == _host_ws_mirror(*shape, 4)
+    assert hw(*shape, 1) == _host_ws_mirror(*shape, 2)
+    assert hw(*shape, 2) == 0                                   # no such output type
+    # a fraction of what mxattn_forward holds on the device (bf16 Q, K, V, fp32 output, workspace)
+    B, Hq, Hkv, N, d = shape
+    if Hkv >= 8:
+        resident = (2 * B * (Hq + 2 * Hkv) + 4 * B * Hq) * N * d + lib.mxattn_forward_workspace_size(*shape)
+        assert hw(*shape, 0) < resident / 4
+
+
+def test_host_forward_argument_checks(lib):
+    f = lib.mxattn_forward_host
+    good = lib.mxattn_forward_host_workspace_size(1, 2, 2, 256, 64, 0)
+
+    def call(q=FAKE, out=FAKE, Hq=2, d=64, mode=1, od=0, wsb=good):
+        return f(q, FAKE, FAKE, out, 1, Hq, 2, 256, d, 0, mode, 1, od, FAKE, wsb, None)
+
+    assert call(q=None) == INVALID
+    assert call(out=None) == INVALID
+    assert call(Hq=3) == INVALID
+    assert call(mode=3) == INVALID
+    assert call(od=5) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(wsb=good - 1) == WORKSPACE
+
+
 def test_forward_argument_checks(lib):
     f = lib.mxattn_forward
     good = lib.mxattn_forward_workspace_size(1, 2, 2, 256, 64)

@@ -36,3 +36,30 @@ def test_host_pipeline_matches_forward(dev, name, mode, out_dtype):
     ref = api.mxattn_forward(q.to(dev), k.to(dev), v.to(dev), causal=cfg.causal, scale_mode=mode,
                              out_dtype=out_dtype).cpu()
     assert torch.equal(out_h, ref)
+
+
+def test_host_pipeline_is_ordered_on_the_callers_stream(dev):
+    """The call runs on side streams of its own, but it must start after, and finish before, the
+    work around it on the caller's stream. Here the pinned inputs are filled by copies queued on a
+    non-default stream just before each call, two calls with different inputs share one
+    workspace, and the outputs are read after that stream alone has been synchronised."""
+    cfg = synthetic.ATTN_CONFIGS["llm_gqa"].scaled(B=2, N=4096)       # chunks of 2, 4, 4, 4, 2 KV heads
+    q, k, v = synthetic.attn_inputs(cfg)
+    q2, k2, v2 = (-t for t in (q, k, v))
+    n = api._lib.load().mxattn_forward_host_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.d, 0)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    dev_inputs = [tuple(t.to(dev) for t in x) for x in ((q, k, v), (q2, k2, v2))]
+    pinned = [tuple(torch.zeros(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)) for _ in range(2)]
+    outs = [torch.zeros(q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    side = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(side):
+        for i in range(2):
+            for h, d_ in zip(pinned[i], dev_inputs[i]):
+                h.copy_(d_, non_blocking=True)
+            api.mxattn_forward_host(*pinned[i], outs[i], causal=cfg.causal, workspace=ws, device=dev)
+    side.synchronize()
+    for i in range(2):
+        ref = api.mxattn_forward(*dev_inputs[i], causal=cfg.causal).cpu()
+        assert torch.equal(outs[i], ref), i
+    assert api.mxattn_check_status(ws) == 0
