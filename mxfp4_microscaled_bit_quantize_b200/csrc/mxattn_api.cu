@@ -613,10 +613,10 @@ mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, v
   const size_t hd = static_cast<size_t>(N) * d;
   const size_t out_elem = (out_dtype == MXATTN_OUT_F32) ? 4 : 2;
 
-  // events: start (orders the side streams after earlier work on the caller's stream), and per
-  // chunk inputs-in, inputs-consumed, compute-done, output-out
+  // events: start (orders the side streams after earlier work on the caller's stream); per chunk
+  // inputs-in, inputs-consumed, compute-done, output-out; and one tail per side stream
   const int chunks = static_cast<int>(P.sizes.size());
-  std::vector<cudaEvent_t> ev(1 + 4 * static_cast<size_t>(chunks), nullptr);
+  std::vector<cudaEvent_t> ev(4 + 4 * static_cast<size_t>(chunks), nullptr);
   for (auto& e : ev)
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) s = MXATTN_ERR_CUDA;
   auto ev_in = [&](int c) { return ev[1 + 4 * c]; };
@@ -669,9 +669,14 @@ mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, v
     ok(cudaMemcpyAsync(static_cast<uint8_t*>(out) + q_off * out_elem, dout, ob, cudaMemcpyDeviceToHost, ss.out));
     ok(cudaEventRecord(ev_out(c), ss.out));
   }
-  // the call completes on the caller's stream once the last output has been copied out (each
-  // copy-out waited for its chunk's kernels, and the copy-out stream runs in chunk order)
-  if (s == MXATTN_OK) ok(cudaStreamWaitEvent(st, ev_out(chunks - 1), 0));
+  // the call completes on the caller's stream once everything it queued on the side streams has
+  // run, on an error path too, so that the caller may free the buffers once its stream is done
+  cudaStream_t side[3] = {ss.in, ss.comp, ss.out};
+  for (int i = 0; i < 3; ++i) {
+    cudaEvent_t tail = ev[1 + 4 * static_cast<size_t>(chunks) + i];
+    if (tail && cudaEventRecord(tail, side[i]) == cudaSuccess) ok(cudaStreamWaitEvent(st, tail, 0));
+    else if (s == MXATTN_OK) s = MXATTN_ERR_CUDA;
+  }
   for (auto& e : ev)
     if (e) cudaEventDestroy(e);   // released once recorded work completes
   return s;
