@@ -67,7 +67,9 @@ def profile_traffic(name: str, src_hash: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms during the timed region. The
+    sampler starts first; entering returns once its first sample has arrived (or after 3 s), and
+    only the samples that arrive between entry and exit are summarised (all of them if none do)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -75,26 +77,48 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.samples = []        # (arrival time, line)
+        self.lines = []
+        self.in_region = False
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.monotonic(), ln))
 
     def __enter__(self):
+        import shutil
+        import threading
+        cmd = ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if shutil.which("stdbuf"):
+            cmd = ["stdbuf", "-oL"] + cmd      # one line per sample as it is taken
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        if self.proc is not None:
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            deadline = time.monotonic() + 3.0
+            while not self.samples and self.proc.poll() is None and time.monotonic() < deadline:
+                time.sleep(0.01)
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        t1 = time.monotonic()
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=5)
+        inside = [ln for t, ln in self.samples if self.t0 <= t <= t1]
+        self.in_region = bool(inside)
+        self.lines = inside or [ln for _, ln in self.samples]
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -112,7 +136,8 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "timed region" if self.in_region else "around the timed region"}
 
 
 def reduce_max_over_ranks(values, world: int, device=None):
