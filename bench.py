@@ -26,6 +26,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "video_dit"
+OTHER_CONFIGS = ("video_dit_long", "llm_gqa")   # also timed, attention per step (UOS + PNQ)
 METRIC = "MXFP4 attention fwd TFLOP/s (video-DiT 1x40x32760x128, UOS+PNQ)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 FP4_PER_BF16 = 4.0          # nominal dense ratio: 9 PFLOP/s fp4 vs 2.25 PFLOP/s bf16
@@ -359,6 +360,39 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         raise RuntimeError("device pipeline timeout in the NVFP4 attention")
     nv_attn_ms = n_start.elapsed_time(n_stop) / fq_steps
 
+    # the other full-size attention workloads: the long video DiT and the causal GQA prefill
+    # (quantizers + attention kernel per step, timed per phase as in the main loop)
+    other = {}
+    for name in OTHER_CONFIGS:
+        ocfg = synthetic.ATTN_CONFIGS[name]
+        oq, ok_, ov = (t.to(dev) for t in synthetic.attn_inputs(ocfg))
+        o_ws = api.alloc_workspace(ocfg.B, ocfg.Hq, ocfg.Hkv, ocfg.N, ocfg.d, dev)
+        o_out = torch.empty((ocfg.B, ocfg.Hq, ocfg.N, ocfg.d), dtype=torch.float32, device=dev)
+
+        def o_step(e=None):
+            if e is not None:
+                e[0].record(stream)
+            api.mxattn_forward_prepare(oq, ok_, ov, api.SCALE_UOS, o_ws)
+            if e is not None:
+                e[1].record(stream)
+            api.mxattn_forward_attend(o_out, ocfg.B, ocfg.Hq, ocfg.Hkv, ocfg.N, ocfg.d, ocfg.causal, api.SCALE_UOS,
+                                      True, o_ws)
+            if e is not None:
+                e[2].record(stream)
+
+        for _ in range(3):
+            o_step()
+        barrier()
+        o_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(fq_steps)]
+        for e in o_ev:
+            o_step(e)
+        barrier()
+        if api.mxattn_check_status(o_ws) != 0:
+            raise RuntimeError(f"device pipeline timeout on {name}")
+        other[name] = (ocfg, float(np.mean([e[1].elapsed_time(e[2]) for e in o_ev])),
+                       float(np.mean([e[0].elapsed_time(e[2]) for e in o_ev])))
+        del oq, ok_, ov, o_ws, o_out
+
     # block-scaled MXFP4 GEMM (W4A4) on its own workload: A [M, K], B [N, K] quantized once
     gm, gn, gk = synthetic.GEMM_SHAPE
     ga = torch.randn((gm, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(5))
@@ -411,9 +445,11 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     del qbuf
 
     # max over ranks
+    other_ms = [x for name in OTHER_CONFIGS for x in other[name][1:]]
     (step_ms, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
-     nv_attn_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms,
-                                          fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms], world, dev)
+     nv_attn_ms, *other_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, copy_ms,
+                                                     quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms,
+                                                     *other_ms], world, dev)
     if rank != 0:
         return
 
@@ -456,6 +492,13 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                             "note": "MXATTN_SCALE_NVFP4 (Q, K, V, P~ in NVFP4), attention kernel alone"},
         "forward_quantized": {"ms": fq_ms, "tflops": flops / (fq_ms * 1e-3) / 1e12,
                               "note": "mxattn_forward_quantized on pre-quantized Q/K/V: scale repack + kernel"},
+        "other_configs": {
+            name: {"workload": other[name][0].describe(), "attn_ms": other_ms[2 * i],
+                   "tflops": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12,
+                   "frac": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12 / fp4_peak,
+                   "step_ms": other_ms[2 * i + 1],
+                   "step_tflops": other[name][0].flops / (other_ms[2 * i + 1] * 1e-3) / 1e12}
+            for i, name in enumerate(OTHER_CONFIGS)},
         "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
                  "tflops": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12,
                  "frac": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12 / fp4_peak,
