@@ -221,7 +221,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     build.build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synthetic.ATTN_CONFIGS[WORKLOAD]
+    cfg = synthetic.ATTN_CONFIGS[args.workload]
     if args.heads:
         cfg = cfg.scaled(Hq=args.heads, Hkv=args.heads)
     B, Hq, Hkv, N, d = cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.d
@@ -594,7 +594,11 @@ def main():
     ap.add_argument("--mode", choices=["full", "attention", "quantizer", "gemm"], default="full",
                     help="attention / quantizer: time only that part (small cases for profiling)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
+    ap.add_argument("--workload", choices=[WORKLOAD, *OTHER_CONFIGS], default=WORKLOAD,
+                    help="the attention workload of --mode attention (profiling only)")
     args = ap.parse_args()
+    if args.workload != WORKLOAD and (args.mode != "attention" or args.heads):
+        ap.error("--workload applies to --mode attention, without --heads")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
