@@ -244,9 +244,11 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
+    mode = {"uos": api.SCALE_UOS, "ocp": api.SCALE_OCP, "nvfp4": api.SCALE_NVFP4}[args.scale]
+
     def step():
-        api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_UOS, ws)
-        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, True, ws)
+        api.mxattn_forward_prepare(dq, dk, dv, mode, ws)
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, True, ws)
 
     for _ in range(args.warmup):
         step()
@@ -260,9 +262,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_UOS, ws)
+            api.mxattn_forward_prepare(dq, dk, dv, mode, ws)
             ev[i][1].record(stream)
-            api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, True, ws)
+            api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, True, ws)
             ev[i][2].record(stream)
         stop.record(stream)
         barrier()
@@ -272,7 +274,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     quant_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
     if args.mode == "attention":
-        print(json.dumps({"mode": "attention", "config": cfg.describe(), "attn_ms": attn_ms,
+        print(json.dumps({"mode": "attention", "scale": args.scale, "config": cfg.describe(), "attn_ms": attn_ms,
                           "quant_ms": quant_ms, "tflops": cfg.flops / (attn_ms * 1e-3) / 1e12}), flush=True)
         return
 
@@ -489,7 +491,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                       "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
         "nvfp4_attention": {"ms": nv_attn_ms, "tflops": flops / (nv_attn_ms * 1e-3) / 1e12,
-                            "note": "MXATTN_SCALE_NVFP4 (Q, K, V, P~ in NVFP4), attention kernel alone"},
+                            "note": "MXATTN_SCALE_NVFP4 (Q, K, V, P~ in NVFP4), attention kernel alone",
+                            "traffic": profile_traffic("attn_fwd_video_dit_nvfp4.json", sources_hash(ATTN_SOURCES))},
         "forward_quantized": {"ms": fq_ms, "tflops": flops / (fq_ms * 1e-3) / 1e12,
                               "note": "mxattn_forward_quantized on pre-quantized Q/K/V: scale repack + kernel"},
         "other_configs": {
@@ -497,7 +500,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                    "tflops": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12,
                    "frac": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12 / fp4_peak,
                    "step_ms": other_ms[2 * i + 1],
-                   "step_tflops": other[name][0].flops / (other_ms[2 * i + 1] * 1e-3) / 1e12}
+                   "step_tflops": other[name][0].flops / (other_ms[2 * i + 1] * 1e-3) / 1e12,
+                   "traffic": profile_traffic(f"attn_fwd_{name}.json", sources_hash(ATTN_SOURCES))}
             for i, name in enumerate(OTHER_CONFIGS)},
         "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
                  "tflops": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12,
@@ -596,9 +600,13 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
     ap.add_argument("--workload", choices=[WORKLOAD, *OTHER_CONFIGS], default=WORKLOAD,
                     help="the attention workload of --mode attention (profiling only)")
+    ap.add_argument("--scale", choices=["uos", "ocp", "nvfp4"], default="uos",
+                    help="the scale mode of --mode attention (profiling only)")
     args = ap.parse_args()
     if args.workload != WORKLOAD and (args.mode != "attention" or args.heads):
         ap.error("--workload applies to --mode attention, without --heads")
+    if args.scale != "uos" and args.mode != "attention":
+        ap.error("--scale applies to --mode attention")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
