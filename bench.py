@@ -176,6 +176,58 @@ def oracle_sample(cfg, rows: int, head: int = 0):
     return flops, dt
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_tiny_full():
+    """The whole tiny workload (1x2x256x64, UOS + PNQ) through the oracle: (FLOP, seconds)."""
+    from mxfp4_microscaled_bit_quantize_b200 import synthetic
+    from oracle import attention as oa
+    from oracle import mxfp4 as mx
+    cfg = synthetic.ATTN_CONFIGS["tiny"]
+    q, k, v = (t.double().numpy() for t in synthetic.attn_inputs(cfg))
+    t0 = time.perf_counter()
+    oa.mxattention(q, k, v, causal=cfg.causal, mode=mx.SCALE_UOS, pnq=True)
+    return cfg.flops, time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, rows: int) -> dict:
+    """The CPU oracle as it stands on this host: a bounded row sample of the workload (rows are
+    independent under the online softmax, so the sample is exact for those rows), its linear
+    extrapolation to the whole workload, the tiny workload in full, and one thread on a smaller
+    sample."""
+    f, dt = oracle_sample(cfg, rows)
+    threads = blas_threads()
+    out = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+           "sample": f"{rows} query rows of head 0 (that head's Q/K/V quantized, attention over all "
+                     f"{cfg.N} keys), {dt:.1f} s",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count(), "blas_threads": threads,
+           "extrapolated": {"seconds": cfg.flops / (f / dt),
+                            "note": f"the sample's rate scaled to all {cfg.B * cfg.Hq * cfg.N} query rows "
+                                    f"of {cfg.name} (extrapolated, not run)"}}
+    tf, tdt = oracle_tiny_full()
+    out["tiny_full"] = {"seconds": tdt, "value": tf / tdt / 1e12, "unit": "TFLOP/s",
+                        "workload": "tiny 1x2x256x64, UOS+PNQ, every row (run in full)"}
+    try:   # the same oracle on one thread (BLAS limited to 1), on an eighth of the rows
+        from threadpoolctl import threadpool_limits
+        rows1 = max(64, rows // 8)
+        with threadpool_limits(limits=1):
+            f1, dt1 = oracle_sample(cfg, rows1)
+        out["single_thread"] = {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s", "rows": rows1, "seconds": dt1}
+    except ImportError:
+        pass
+    return out
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -207,7 +259,10 @@ def run_reference(args, rank: int) -> None:
             "data": "synthetic", "config": {"workload": WORKLOAD, **cfg.describe(), "scale_mode": "UOS",
                                             "pnq": True, "sample_rows": rows},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                             "extrapolated": {"seconds": cfg.flops / (flops / secs),
+                                              "note": "the sample's rate scaled to the whole workload "
+                                                      "(extrapolated, not run)"}},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -395,13 +450,12 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                        float(np.mean([e[0].elapsed_time(e[2]) for e in o_ev])))
         del oq, ok_, ov, o_ws, o_out
 
-    # block-scaled MXFP4 GEMM (W4A4) on its own workload: A [M, K], B [N, K] quantized once
+    # block-scaled MXFP4 GEMM (W4A4) on its own seeded workload (the one its parity test samples):
+    # A [M, K] activations with per-row gains, B [N, K] weights, quantized once outside the timing
     gm, gn, gk = synthetic.GEMM_SHAPE
-    ga = torch.randn((gm, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(5))
-    gb = torch.randn((gn, gk), device=dev, dtype=torch.float32, generator=torch.Generator(dev).manual_seed(6))
-    g_ops = (*api.mxattn_quantize(ga.bfloat16(), False, api.SCALE_UOS),
-             *api.mxattn_quantize((gb * 0.05).bfloat16(), False, api.SCALE_UOS))
-    nv_ops = (*api.mxattn_quantize_nvfp4(ga.bfloat16()), *api.mxattn_quantize_nvfp4((gb * 0.05).bfloat16()))
+    ga, gb = (t.to(dev) for t in synthetic.gemm_inputs(gm, gn, gk))
+    g_ops = (*api.mxattn_quantize(ga, False, api.SCALE_UOS), *api.mxattn_quantize(gb, False, api.SCALE_UOS))
+    nv_ops = (*api.mxattn_quantize_nvfp4(ga), *api.mxattn_quantize_nvfp4(gb))
     del ga, gb
     g_ws = api.gemm_workspace(gm, gn, gk, dev)
     g_out = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
@@ -430,21 +484,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     gemm_nv_ms = g_start.elapsed_time(g_stop) / g_iters
     del g_ops, nv_ops, g_ws, g_out
 
-    # standalone quantizer on its own workload (65536 x 1024 bf16), two buffer sets > L2
-    xq = [synthetic.quant_input().to(dev) for _ in range(2)]
-    qbuf = [api.mxattn_quantize(x, False, api.SCALE_UOS) for x in xq]
-    for i in range(5):
-        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
-    barrier()
-    qs, qe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    qiters = 50
-    qs.record(stream)
-    for i in range(qiters):
-        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
-    qe.record(stream)
-    barrier()
-    quant_alone_ms = qs.elapsed_time(qe) / qiters
-    del qbuf
+    # standalone quantizer on its own workload (65536 x 1024 bf16)
+    quant_alone_ms, xq0_numel = time_quantizer_rotating(dev, stream, barrier, iters=50)
 
     # max over ranks
     other_ms = [x for name in OTHER_CONFIGS for x in other[name][1:]]
@@ -462,7 +503,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     elems = B * Hq * N * d + 2 * B * Hkv * N * d
     # algorithmic bytes of the three quantizer launches: bf16 in, packed codes + scales out
     quant_bytes = elems * 2 + elems // 2 + elems // 32
-    qa_elems = xq[0].numel()
+    qa_elems = xq0_numel
     qa_bytes = qa_elems * 2 + qa_elems // 2 + qa_elems // 32
     line = {
         "metric": METRIC,
@@ -488,6 +529,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "quantizer": {"in_step_gbs": quant_bytes / (quant_ms * 1e-3) / 1e9, "in_step_ms": quant_ms,
                       "standalone_65536x1024_gbs": qa_bytes / (quant_alone_ms * 1e-3) / 1e9,
                       "standalone_ms": quant_alone_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
+                      "standalone_buffers": f"{QUANT_SETS} input/output sets rotated, "
+                                            f"{QUANT_SETS * qa_bytes / 1e6:.0f} MB in all (> 2 x 126 MB L2)",
                       "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
         "nvfp4_attention": {"ms": nv_attn_ms, "tflops": flops / (nv_attn_ms * 1e-3) / 1e12,
@@ -521,20 +564,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:
-        f, dt = oracle_sample(cfg, args.cpu_rows)
-        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-                                "kind": "oracle",
-                                "sample": f"{args.cpu_rows} query rows of head 0 (that head's Q/K/V "
-                                          f"quantized, attention over all {cfg.N} keys), {dt:.1f} s"}
-        try:   # the same oracle on one thread (BLAS limited to 1), on an eighth of the rows
-            from threadpoolctl import threadpool_limits
-            rows1 = max(64, args.cpu_rows // 8)
-            with threadpool_limits(limits=1):
-                f1, dt1 = oracle_sample(cfg, rows1)
-            line["cpu_baseline"]["single_thread"] = {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s", "rows": rows1,
-                                                     "seconds": dt1}
-        except ImportError:
-            pass
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_rows)
     print(json.dumps(line), flush=True)
 
 
@@ -546,8 +576,7 @@ def run_gemm_only(args, dev):
     gm, gn, gk = synthetic.GEMM_SHAPE
     if args.heads:
         gm = 128 * args.heads
-    ga = torch.randn((gm, gk), device=dev, generator=torch.Generator(dev).manual_seed(5)).bfloat16()
-    gb = (torch.randn((gn, gk), device=dev, generator=torch.Generator(dev).manual_seed(6)) * 0.05).bfloat16()
+    ga, gb = (t.to(dev) for t in synthetic.gemm_inputs(gm, gn, gk))
     ops = (*api.mxattn_quantize(ga, False, api.SCALE_UOS), *api.mxattn_quantize(gb, False, api.SCALE_UOS))
     ws = api.gemm_workspace(gm, gn, gk, dev)
     out = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
@@ -565,23 +594,37 @@ def run_gemm_only(args, dev):
                       "tflops": 2.0 * gm * gn * gk / (ms * 1e-3) / 1e12}), flush=True)
 
 
-def run_quantizer_only(args, dev):
-    """The standalone quantizer workload alone (used for its Nsight Compute capture)."""
+QUANT_SETS = 4      # input/output buffer sets the standalone quantizer rotates through
+
+
+def time_quantizer_rotating(dev, stream, barrier, iters: int, warmup: int = 5):
+    """Mean ms per call of the standalone quantizer (65536 x 1024, UOS) on QUANT_SETS sets of input
+    and output buffers used in turn, so that neither the bf16 input nor the codes and scales written
+    by one call are still in L2 when their set comes round again (4 x 170 MB > 2 x 126 MB L2)."""
     import torch
 
     from mxfp4_microscaled_bit_quantize_b200 import api, synthetic
-    xq = [synthetic.quant_input().to(dev) for _ in range(2)]
-    for i in range(args.warmup):
-        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
-    torch.cuda.synchronize(dev)
+    x0 = synthetic.quant_input().to(dev)
+    xs = [x0] + [x0.clone() for _ in range(QUANT_SETS - 1)]
+    outs = [api.mxattn_quantize(x, False, api.SCALE_UOS) for x in xs]
+    for i in range(warmup):
+        api.mxattn_quantize(xs[i % QUANT_SETS], False, api.SCALE_UOS, out=outs[i % QUANT_SETS])
+    barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for i in range(args.steps):
-        api.mxattn_quantize(xq[i % 2], False, api.SCALE_UOS)
-    e.record()
-    torch.cuda.synchronize(dev)
-    ms = s.elapsed_time(e) / args.steps
-    n = xq[0].numel()
+    s.record(stream)
+    for i in range(iters):
+        api.mxattn_quantize(xs[i % QUANT_SETS], False, api.SCALE_UOS, out=outs[i % QUANT_SETS])
+    e.record(stream)
+    barrier()
+    return s.elapsed_time(e) / iters, x0.numel()
+
+
+def run_quantizer_only(args, dev):
+    """The standalone quantizer workload alone (used for its Nsight Compute capture)."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    ms, n = time_quantizer_rotating(dev, stream, lambda: torch.cuda.synchronize(dev), iters=args.steps,
+                                    warmup=args.warmup)
     gbs = (n * 2 + n // 2 + n // 32) / (ms * 1e-3) / 1e9
     print(json.dumps({"mode": "quantizer", "ms": ms, "gbs": gbs}), flush=True)
 

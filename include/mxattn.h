@@ -29,7 +29,11 @@
  * Conventions
  * -----------
  *   - Every pointer argument named as device memory must be a CUDA device pointer on the
- *     current device. The caller owns every buffer; the library never allocates device memory.
+ *     current device. The caller owns every buffer it passes, and no entry point calls
+ *     cudaMalloc. Two exceptions hold library-owned resources: every device that loads the
+ *     library reserves a fixed MXATTN_NOALLOC_MAX_WORKSPACE-byte static array (the workspace of
+ *     mxattn_forward_noalloc) when the library's device module is loaded, and
+ *     mxattn_forward_host creates its own streams and events on first use.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are asynchronous on it.
  *   - Argument errors are detected on the host and returned before anything is launched.
  *     Launch errors return MXATTN_ERR_CUDA. A device-side pipeline timeout (every wait inside
@@ -235,13 +239,19 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
  * q, k, v and out exactly as for mxattn_forward; the workspace instead comes from a static
  * device array of MXATTN_NOALLOC_MAX_WORKSPACE bytes that every GPU loading the library holds
  * until the process exits.
- *   - Shapes with mxattn_forward_workspace_size(...) > MXATTN_NOALLOC_MAX_WORKSPACE are rejected
- *     with MXATTN_ERR_WORKSPACE before anything is launched.
- *   - The first call on a device (that device current) looks up the array's device address;
- *     make it before any stream capture. No call allocates.
+ *   - Every argument is checked exactly as mxattn_forward checks it when handed a workspace of
+ *     MXATTN_NOALLOC_MAX_WORKSPACE bytes: shapes with mxattn_forward_workspace_size(...) larger
+ *     than that get MXATTN_ERR_WORKSPACE, every other rejected call the code mxattn_forward
+ *     returns, all before anything is launched. No call allocates.
+ *   - Each call looks up the array's device address in the current context (so it stays valid
+ *     after cudaDeviceReset or in a non-primary context). The first call in a context may load
+ *     the library's device module: make it before any stream capture.
  *   - All calls on a device share the array: calls whose kernels overlap on the GPU race, so
  *     serialise them (one stream, or explicit ordering). The status word is cleared at the
- *     start of each call; device-side timeouts are not reported by this entry point.
+ *     start of each call. A device-side wait timeout is recorded only in the shared array,
+ *     which no caller can read: the call has already returned MXATTN_OK and `out` is then
+ *     unspecified. Callers that must detect timeouts use mxattn_forward with their own
+ *     workspace and mxattn_check_status.
  */
 #define MXATTN_NOALLOC_MAX_WORKSPACE ((size_t)16 << 20)
 mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq,

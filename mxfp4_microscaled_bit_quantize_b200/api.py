@@ -33,11 +33,12 @@ def npad(N: int) -> int:
     return -(-N // NPAD_ALIGN) * NPAD_ALIGN
 
 
-def mxattn_quantize(x: torch.Tensor, transpose: bool = False, scale_mode: int = SCALE_UOS):
+def mxattn_quantize(x: torch.Tensor, transpose: bool = False, scale_mode: int = SCALE_UOS, out=None):
     """MXFP4-quantize the last two axes [rows, cols] of a bf16 CUDA tensor.
 
     transpose=False: blocks of 32 along cols -> codes [..., rows, ceil(cols/32)*16], scales [..., rows, ceil(cols/32)].
     transpose=True:  blocks of 32 along rows -> codes [..., cols, ceil(rows/32)*16], scales [..., cols, ceil(rows/32)].
+    out: optional (codes, scales) uint8 CUDA tensors of exactly those shapes, written in place.
     """
     _need(x, "x")
     if x.dim() < 2:
@@ -45,14 +46,17 @@ def mxattn_quantize(x: torch.Tensor, transpose: bool = False, scale_mode: int = 
     lead = tuple(x.shape[:-2])
     rows, cols = int(x.shape[-2]), int(x.shape[-1])
     batch = math.prod(lead) if lead else 1
-    if transpose:
-        nb = -(-rows // 32)
-        codes = torch.empty(lead + (cols, nb * 16), dtype=torch.uint8, device=x.device)
-        scales = torch.empty(lead + (cols, nb), dtype=torch.uint8, device=x.device)
+    nb = -(-(rows if transpose else cols) // 32)
+    outer = cols if transpose else rows
+    if out is None:
+        codes = torch.empty(lead + (outer, nb * 16), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lead + (outer, nb), dtype=torch.uint8, device=x.device)
     else:
-        nb = -(-cols // 32)
-        codes = torch.empty(lead + (rows, nb * 16), dtype=torch.uint8, device=x.device)
-        scales = torch.empty(lead + (rows, nb), dtype=torch.uint8, device=x.device)
+        codes, scales = out
+        for t, shape, name in ((codes, lead + (outer, nb * 16), "codes"), (scales, lead + (outer, nb), "scales")):
+            _need(t, name, torch.uint8)
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
     lib = _lib.load()
     st = lib.mxattn_quantize(x.data_ptr(), batch, rows, cols, int(bool(transpose)), int(scale_mode),
                              codes.data_ptr(), scales.data_ptr(), _stream(x.device))
