@@ -57,7 +57,7 @@ typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1, MXATTN_SCALE_NVFP4 = 
 
 /* Keys per tile of the online softmax. P~ is quantized with the running max in force at each
  * tile, so the tile width is part of the result (a CPU reference must use the same width). */
-#define MXATTN_KV_TILE 64
+#define MXATTN_KV_TILE 128
 
 typedef enum { MXATTN_OUT_F32 = 0, MXATTN_OUT_BF16 = 1 } mxattn_out_dtype;
 

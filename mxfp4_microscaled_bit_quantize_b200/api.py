@@ -12,7 +12,7 @@ from . import _lib
 
 SCALE_OCP, SCALE_UOS, SCALE_NVFP4 = 0, 1, 2
 OUT_F32, OUT_BF16 = 0, 1
-KV_TILE = 64          # keys per online-softmax tile (MXATTN_KV_TILE)
+KV_TILE = 128         # keys per online-softmax tile (MXATTN_KV_TILE)
 NPAD_ALIGN = 128      # the workspace pads N to a multiple of this
 
 

@@ -13,23 +13,29 @@
 //   pnq = 0 keeps the conventional path: l sums the unquantized fp32 P~ on the CUDA cores.
 //   out = O / l.
 //
-// One CTA owns one 128-query tile of one (batch, query head) and visits keys in tiles of
-// kKvTile = 64 in increasing order (P~ codes depend on the running max in force, so tile width
-// and order are part of the definition; the oracle takes the same width). Two CTAs share an SM:
-// each allocates half of TMEM and their softmax phases drift apart, so one CTA's exponentials
-// overlap the other's serial work (max, scale selection, stores, rescale).
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q tile once, then K / V^T tiles and their scale atoms into an
-//              NSTAGE-deep shared-memory ring (mbarrier complete_tx).
-//   warp 1     TMEM owner and MMA issuer (one thread): copies scale atoms to TMEM with
-//              tcgen05.cp, issues S = QK^T, O += P~ V^T and (PNQ) L += P~ 1.
-//   warps 2-5  softmax warpgroup, one thread per query row (TMEM lane = row): reads S with
-//              tcgen05.ld (S is single-buffered: the MMA for the next tile starts as soon as the
-//              row is in registers), updates the running max, computes P~ / 2^e per 32-key block,
-//              quantizes it in registers, writes codes (32B-swizzled, the MMA operand layout)
-//              and scale bytes to shared memory, rescales O and L in TMEM when the max moves,
-//              and finally normalises and stores the output.
-// TMEM (256 columns per CTA): S [0,64) O [64,64+d) L [192,208) scale atoms 208..243.
+// Work unit: one CTA (one per SM: it allocates all 512 TMEM columns) owns two consecutive
+// 128-query tiles A and B of one (batch, query head) and visits keys in tiles of kKvTile = 128 in
+// increasing order (P~ codes depend on the running max in force, so tile width and order are part
+// of the definition; the oracle takes the same width). The two query tiles share every K / V^T
+// tile in shared memory and take turns on ONE 128-column S buffer in TMEM: S(A, t), S(B, t),
+// S(A, t+1), ... . Their softmax warps therefore run half a step apart, and on every SM
+// sub-partition one tile's serial work (S load, maxima, scale selection, stores, rescale) overlaps
+// the other tile's exponentials on the MUFU.
+// Warp roles (320 threads):
+//   warp 0     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
+//              an NSTAGE-deep shared-memory ring (mbarrier complete_tx).
+//   warp 1     TMEM owner and MMA issuer (one thread): copies scale atoms to TMEM with tcgen05.cp
+//              and issues, per key tile t, S(A, t+1), O_A += P~_A(t) V(t) (+ L_A), S(B, t+1),
+//              O_B += P~_B(t) V(t) (+ L_B). Each S waits until the previous user of the S buffer
+//              holds its scores in registers.
+//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one thread per query row (TMEM lane = row).
+//              Per key tile a thread reads its 128 scores with tcgen05.ld, releases S, updates the
+//              running max, computes P~ / 2^e per 32-key block, quantizes it in registers, writes
+//              64 bytes of codes (64B-swizzled, the MMA operand layout) and four scale bytes to
+//              shared memory, rescales O and L in TMEM when the max moves, and at the end
+//              normalises and stores the output row.
+// TMEM (512 columns): S [0,128) O_A [128,128+d) O_B [256,256+d) L_A [384,400) L_B [400,416),
+// scale atoms from 416 (see kColSf*).
 // The kernel is templated on the format: MXFP4 (the method) or, for comparison, NVFP4 (blocks of
 // 16 with E4M3 scales for Q, K, V and P~; kind::mxf4nvf4 products, the non-power-of-two P~ scale
 // folded into the exponent bias as -log2 s).
@@ -42,58 +48,59 @@
 
 namespace mxattn {
 
-constexpr int kBM = 128;          // query rows per CTA
-constexpr int kBN = kKvTile;      // keys per KV tile (64)
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 64, kColL = 192;
-// Q and K scale atoms: one per 64 (NVFP4) or 128 (MXFP4) contraction elements, 4 columns each.
-constexpr uint32_t kColSfQ = 208, kColSfK = 216, kColSf1 = 224;
-// P~ scale atoms alternate between two column sets by tile parity, V scale atoms (one per pair of
-// 64-key tiles) by pair parity: tcgen05.cp into columns an earlier MMA still reads is not ordered
-// behind that MMA, and the product of tile j may still run when the scales of tile j+1 are
-// copied. The set written for tile j+1 was last read by a product no later than that of tile
-// j-1, which the softmax has seen complete before it hands over tile j+1.
-// NVFP4 gives every 64-key tile its own V atom, which then alternates by tile parity.
-constexpr uint32_t kColSfV = 228, kColSfP = 236;   // + 4 * set
+constexpr int kBM = 128;          // query rows per Q tile (the MMA's M)
+constexpr int kBN = kKvTile;      // keys per KV tile (128)
+constexpr int kSoftmaxWarps = 8;  // four per query tile
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;   // 320: producer, MMA, softmax A, softmax B
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 X, L_X at kColL + 16 X
+// Scale atoms, 4 columns each (NVFP4 needs two per operand tile, MXFP4 one):
+//   Q_X         kColSfQ + 8 X
+//   K of tile t kColSfK + 8 (t & 1)      V of tile t kColSfV + 8 (t & 1)
+//   P~_X(t)     kColSfP + 16 X + 8 (t & 1)
+//   ones        kColSf1
+// tcgen05.cp into columns an earlier MMA still reads is not ordered behind that MMA; the K, V and
+// P~ sets alternate by tile parity, and the set written for tile t was last read by a product of
+// tile t - 2, which the issuing thread has seen complete by then (see the MMA issuer).
+constexpr uint32_t kColSfQ = 416, kColSfK = 432, kColSfV = 448, kColSfP = 464, kColSf1 = 496;
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
-constexpr int kPRowBytes = kBN / 2;                  // 32 bytes of codes per P~ row
-constexpr size_t kMinSmem = 80 * 1024;               // at most two CTAs per SM (TMEM halves)
+constexpr int kPRowBytes = kBN / 2;                  // 64 bytes of codes per P~ / V^T row
 
-static_assert(kBN == 64, "the 32B-swizzled P~ / V^T layouts below assume 64-key tiles");
+static_assert(kBN == 128, "the 64B-swizzled P~ / V^T layouts below assume 128-key tiles");
 
 template <int D>
 struct Cfg {
-  static constexpr int kStages = 8;
+  static constexpr int kStages = (D == 128) ? 6 : 8;
   static constexpr int kQRowBytes = D / 2;                 // packed E2M1 per Q/K row
   static constexpr int kQTileBytes = kBM * kQRowBytes;
   static constexpr int kKTileBytes = kBN * kQRowBytes;
-  static constexpr int kVTileBytes = D * kPRowBytes;       // V^T: D rows of 64 keys
+  static constexpr int kVTileBytes = D * kPRowBytes;       // V^T: D rows of 128 keys
   static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
   static constexpr uint32_t kQKSbo = 8 * kQRowBytes;       // 8-row swizzle atom
 };
 
 template <int D>
 struct __align__(1024) Smem {
-  uint8_t q[Cfg<D>::kQTileBytes];
+  uint8_t q[2][Cfg<D>::kQTileBytes];
   uint8_t k[Cfg<D>::kStages][Cfg<D>::kKTileBytes];
   uint8_t v[Cfg<D>::kStages][Cfg<D>::kVTileBytes];
-  uint8_t p[2][kBM * kPRowBytes];         // P~ codes, double-buffered by tile parity
+  uint8_t p[2][2][kBM * kPRowBytes];      // P~ codes [query tile][tile parity]
   uint8_t ones[kOnesRows * kPRowBytes];
-  uint8_t qsf[1024];                      // MXFP4: one atom; NVFP4: D / 64 atoms
+  uint8_t qsf[2][1024];                   // per query tile: MXFP4 one atom, NVFP4 D / 64 atoms
   uint8_t ksf[Cfg<D>::kStages][1024];
-  uint8_t vsf[Cfg<D>::kStages][512];
-  uint8_t psf[2][512];
+  uint8_t vsf[Cfg<D>::kStages][1024];     // MXFP4 one atom per key tile, NVFP4 two
+  uint8_t psf[2][2][1024];                // [query tile][tile parity]
   uint8_t onesf[512];
   uint64_t bar_q;
   uint64_t bar_kv_full[Cfg<D>::kStages];
   uint64_t bar_kv_empty[Cfg<D>::kStages];
-  uint64_t bar_s_full;
-  uint64_t bar_s_empty;
-  // P~ buffer b written by all 128 rows (tiles of parity b). One barrier per buffer: a fast
-  // softmax warp may arrive for tile j+1 before a slow one has arrived for tile j.
-  uint64_t bar_p_full[2];
-  uint64_t bar_pv_done[2];                 // completions of PV of even / odd tiles
+  uint64_t bar_s_full[2];                 // S of query tile X computed (one phase per key tile)
+  uint64_t bar_s_empty;                   // the S buffer's current user holds it in registers
+  // P~ buffer [X][b] written by the four warps of query tile X (key tiles of parity b). One
+  // barrier per buffer: a fast softmax warp may arrive for tile t+1 before a slow one has arrived
+  // for tile t.
+  uint64_t bar_p_full[2][2];
+  uint64_t bar_pv_done[2][2];             // completions of PV of query tile X, even / odd key tiles
   uint64_t bar_drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -101,7 +108,7 @@ struct __align__(1024) Smem {
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return (sizeof(Smem<D>) + 1024 > kMinSmem) ? sizeof(Smem<D>) + 1024 : kMinSmem;
+  return sizeof(Smem<D>) + 1024;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -158,33 +165,43 @@ __device__ __forceinline__ float lg2_approx(float x) {
 // NV = false: MXFP4 (blocks of 32, UE8M0, OCP or UOS exponent). NV = true: the NVFP4 comparison
 // format for Q, K, V and P~ (blocks of 16, E4M3 scale = RNE(amax / 6)).
 template <int D, bool PNQ, bool DBG, bool NV>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
   constexpr int kQKAtoms = NV ? D / 64 : 1;            // scale atoms per 128 Q or K rows
   constexpr uint32_t kQKSfBytes = kQKAtoms * 512;
+  constexpr int kPVAtoms = NV ? 2 : 1;                 // scale atoms per 128-key V^T or P~ tile
+  constexpr uint32_t kPVSfBytes = kPVAtoms * 512;
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& s = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work tile: (b, kv head g, query head within group, q tile); q tile fastest so that
-  //      co-resident CTAs share one KV head in L2; causal runs the longest tiles first.
+  // ---- work unit: (b, kv head g, query head within group, pair of q tiles); the pair index runs
+  //      fastest so that co-scheduled CTAs share one KV head in L2; causal runs the longest first.
   const int n_qt = p.Npad / kBM;
+  const int n_units = (n_qt + 1) / 2;
   const int group = p.Hq / p.Hkv;
   int idx = blockIdx.x;
-  int qt = idx % n_qt;
-  idx /= n_qt;
+  int unit = idx % n_units;
+  idx /= n_units;
   const int bh_q = idx;                       // b * Hq + h  (h = g * group + hh)
   const int b = idx / p.Hq;
   const int h = idx % p.Hq;
   const int bh_kv = b * p.Hkv + h / group;
-  if (p.causal) qt = n_qt - 1 - qt;
+  if (p.causal) unit = n_units - 1 - unit;
   const int n_kv_all = p.Npad / kBN;
-  const int n_kv = p.causal ? min(2 * qt + 2, n_kv_all) : n_kv_all;
+  int qt_x[2], n_kv_x[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    qt_x[x] = 2 * unit + x;
+    n_kv_x[x] = qt_x[x] >= n_qt ? 0 : (p.causal ? min(qt_x[x] + 1, n_kv_all) : n_kv_all);
+  }
+  const bool has_b = n_kv_x[1] > 0;
+  const int n_kv_max = max(n_kv_x[0], n_kv_x[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(&s.bar_q, 1);
@@ -192,12 +209,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&s.bar_kv_full[i], 1);
       mbar_init(&s.bar_kv_empty[i], 1);
     }
-    mbar_init(&s.bar_s_full, 1);
-    mbar_init(&s.bar_s_empty, kBM);
-    mbar_init(&s.bar_p_full[0], kBM);
-    mbar_init(&s.bar_p_full[1], kBM);
-    mbar_init(&s.bar_pv_done[0], 1);
-    mbar_init(&s.bar_pv_done[1], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s.bar_s_full[x], 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&s.bar_p_full[x][i], 4);      // one arrival per softmax warp of the tile
+        mbar_init(&s.bar_pv_done[x][i], 1);
+      }
+    }
+    mbar_init(&s.bar_s_empty, 4);
     mbar_init(&s.bar_drain, 1);
     s.abort_flag = 0;
     fence_mbar_init();
@@ -220,51 +239,55 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(&s.bar_q, C::kQTileBytes + kQKSfBytes);
-      tma_load_2d(s.q, &tmQ, &s.bar_q, 0, bh_q * p.rows_per_head + qt * kBM);
-      bulk_load(s.qsf, p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt) * kQKSfBytes, kQKSfBytes, &s.bar_q);
+      mbar_arrive_expect_tx(&s.bar_q, (has_b ? 2u : 1u) * (C::kQTileBytes + kQKSfBytes));
+      for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+        tma_load_2d(s.q[x], &tmQ, &s.bar_q, 0, bh_q * p.rows_per_head + qt_x[x] * kBM);
+        bulk_load(s.qsf[x], p.qsf + (static_cast<size_t>(bh_q) * n_qt + qt_x[x]) * kQKSfBytes, kQKSfBytes,
+                  &s.bar_q);
+      }
     }
     __syncwarp();
     int issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j % NS;
-      if (j >= NS) {
-        bool ok = mbar_wait(&s.bar_kv_empty[st], ((j / NS) & 1) ^ 1, abort_flag, p.status,
+    for (int t = 0; t < n_kv_max; ++t) {
+      const int st = t % NS;
+      if (t >= NS) {
+        bool ok = mbar_wait(&s.bar_kv_empty[st], ((t / NS) & 1) ^ 1, abort_flag, p.status,
                             kStatusTimeoutEmpty | st);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (leader) {
-        // K scale atoms cover 128 keys: tiles 2t and 2t+1 share them, loaded with the even tile;
-        // V atoms likewise for MXFP4, one per 64-key tile for NVFP4
-        const bool atoms = (j & 1) == 0;
-        const bool v_atom = NV || atoms;
-        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + (atoms ? kQKSfBytes : 0) +
-                                                      (v_atom ? 512 : 0));
-        tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.rows_per_head + j * kBN);
-        tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], j * kPRowBytes, bh_kv * D);
-        if (atoms)
-          bulk_load(s.ksf[st], p.ksf + (static_cast<size_t>(bh_kv) * n_qt + (j >> 1)) * kQKSfBytes, kQKSfBytes,
-                    &s.bar_kv_full[st]);
-        if (v_atom) {
-          const size_t v_at = NV ? static_cast<size_t>(bh_kv) * (p.Npad / kBN) + j
-                                 : static_cast<size_t>(bh_kv) * n_qt + (j >> 1);
-          bulk_load(s.vsf[st], p.vsf + v_at * 512, 512, &s.bar_kv_full[st]);
-        }
+        mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + kQKSfBytes + kPVSfBytes);
+        tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.rows_per_head + t * kBN);
+        tma_load_2d(s.v[st], &tmV, &s.bar_kv_full[st], t * kPRowBytes, bh_kv * D);
+        bulk_load(s.ksf[st], p.ksf + (static_cast<size_t>(bh_kv) * n_qt + t) * kQKSfBytes, kQKSfBytes,
+                  &s.bar_kv_full[st]);
+        // V^T atoms: MXFP4 one per 128 keys; NVFP4 one per 64 keys, two per key tile
+        const size_t v_at = NV ? static_cast<size_t>(bh_kv) * (p.Npad / 64) + 2 * t
+                               : static_cast<size_t>(bh_kv) * n_qt + t;
+        bulk_load(s.vsf[st], p.vsf + v_at * 512, kPVSfBytes, &s.bar_kv_full[st]);
       }
       __syncwarp();
-      issued = j + 1;
+      issued = t + 1;
     }
     if (*abort_flag && leader) {
       // let every copy this warp started land before the CTA can exit
       drain_wait(&s.bar_q, 0);
-      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-        drain_wait(&s.bar_kv_full[j % NS], (j / NS) & 1);
+      for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
+        drain_wait(&s.bar_kv_full[t % NS], (t / NS) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
     // The whole warp runs the loop (warp-uniform descriptors); one elected lane issues every
     // tcgen05 operation and commit, so completion tracking stays with that thread.
+    //
+    // Order per key tile t: S(A, t+1), PV(A, t), S(B, t+1), PV(B, t). A commit arrives only when
+    // every earlier operation of this thread has completed, so once this thread has seen the
+    // consumer of some S(X, t') (or PV) commit, every operation issued before that one is
+    // complete too. That gives the scale-atom sets their safety: the K set of tile t is written
+    // after the S buffer's previous user read its scores (so the S products of tile t - 2, issued
+    // earlier, are done); the V and P~ sets of tile t are written after PV(X, t)'s softmax has read
+    // S(X, t), which was issued after every product of tile t - 2.
     const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
     auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
     if (PNQ) {
@@ -281,83 +304,97 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok) {
       tc_fence_after();
       if (leader) {
+        for (int x = 0; x < (has_b ? 2 : 1); ++x) {
 #pragma unroll
-        for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfQ + 4 * a, sf_desc(s.qsf + a * 512));
+          for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfQ + 8 * x + 4 * a, sf_desc(s.qsf[x] + a * 512));
+        }
         if (PNQ) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
       }
       __syncwarp();
     }
-    auto issue_s = [&](int j) -> bool {
-      const int st = j % NS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_kv_full[st], (j / NS) & 1, abort_flag, p.status,
-                                             kStatusTimeoutKV | st)))
+    int s_uses = 0;      // S products issued so far (A and B alternate on the one buffer)
+    auto issue_s = [&](int x, int t) -> bool {
+      const int st = t % NS;
+      const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
+      if (first && !__all_sync(0xffffffffu, mbar_wait(&s.bar_kv_full[st], (t / NS) & 1, abort_flag, p.status,
+                                                       kStatusTimeoutKV | st)))
         return false;
-      // S is single-buffered: the previous tile must be in the softmax registers
-      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&s.bar_s_empty, (j - 1) & 1, abort_flag, p.status,
-                                                       kStatusTimeoutS)))
+      // the previous user of the S buffer must hold its scores in registers
+      if (s_uses > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status,
+                                                           kStatusTimeoutS)))
         return false;
       tc_fence_after();
-      const uint32_t qa = smem_u32(s.q), ka = smem_u32(s.k[st]);
-      // keys of an odd tile are rows 64..127 of the scale atom: TMEM columns 2, 3 of it
-      const uint32_t sfk = tmem + kColSfK + 2 * (j & 1);
+      const uint32_t qa = smem_u32(s.q[x]), ka = smem_u32(s.k[st]);
+      const uint32_t sfk = tmem + kColSfK + 8 * (t & 1);
       if (leader) {
-        // the even tile brings the K atoms of the pair; S of the previous pair has completed
-        if ((j & 1) == 0) {
+        if (first) {
 #pragma unroll
-          for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfK + 4 * a, sf_desc(s.ksf[st] + a * 512));
+          for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(sfk + 4 * a, sf_desc(s.ksf[st] + a * 512));
         }
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
           const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
           const uint64_t bd = smem_desc(ka + kk * 32, 0, C::kQKSbo, C::kQKLayout);
           if constexpr (NV)   // one atom (four 16-element blocks) per K = 64 step
-            tc_mma_nvf4(tmem + kColS, ad, bd, idesc_nvf4(kBN), tmem + kColSfQ + 4 * kk, sfk + 4 * kk, kk > 0);
+            tc_mma_nvf4(tmem + kColS, ad, bd, idesc_nvf4(kBN), tmem + kColSfQ + 8 * x + 4 * kk, sfk + 4 * kk, kk > 0);
           else
-            tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ, sfk, kk > 0);
+            tc_mma_mxf4(tmem + kColS, ad, bd, idesc_mxf4(kBN, 2 * kk, 2 * kk), tmem + kColSfQ + 8 * x, sfk, kk > 0);
         }
-        tc_commit(&s.bar_s_full);
+        tc_commit(&s.bar_s_full[x]);
       }
       __syncwarp();
+      ++s_uses;
       return true;
     };
-    auto issue_pv = [&](int j) -> bool {
-      const int st = j % NS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_p_full[j & 1], (j >> 1) & 1, abort_flag, p.status, kStatusTimeoutP)))
+    auto issue_pv = [&](int x, int t) -> bool {
+      const int st = t % NS;
+      const int pb = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status,
+                                             kStatusTimeoutP)))
         return false;
       tc_fence_after();
-      const uint32_t pa = smem_u32(s.p[j & 1]), va = smem_u32(s.v[st]);
-      const uint64_t ad = smem_desc(pa, 0, 8 * kPRowBytes, kLayoutSw32);
-      const uint64_t bd = smem_desc(va, 0, 8 * kPRowBytes, kLayoutSw32);
+      const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
+      const bool last = (x == 1) || t >= n_kv_x[1];       // last reader of the tile's stage
+      const uint32_t pa = smem_u32(s.p[x][pb]), va = smem_u32(s.v[st]);
       if (leader) {
-        const uint32_t sfp = tmem + kColSfP + 4 * (j & 1);
-        const uint32_t sfv = tmem + kColSfV + 4 * (NV ? (j & 1) : ((j >> 1) & 1));
-        tc_cp_sf(sfp, sf_desc(s.psf[j & 1]));
-        if (NV || (j & 1) == 0) tc_cp_sf(sfv, sf_desc(s.vsf[st]));   // MXFP4: the V atom of the tile pair
-        if constexpr (NV) {
-          tc_mma_nvf4(tmem + kColO, ad, bd, idesc_nvf4(D), sfp, sfv, j > 0 ? 1u : 0u);
-          if (PNQ) {
-            const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
-            tc_mma_nvf4(tmem + kColL, ad, od, idesc_nvf4(kOnesRows), sfp, tmem + kColSf1, j > 0 ? 1u : 0u);
-          }
-        } else {
-          // this tile's 64 keys are blocks 0,1 (even tile) or 2,3 (odd tile) of the V scale atom
-          tc_mma_mxf4(tmem + kColO, ad, bd, idesc_mxf4(D, 0, 2 * (j & 1)), sfp, sfv, j > 0 ? 1u : 0u);
-          if (PNQ) {
-            const uint64_t od = smem_desc(smem_u32(s.ones), 0, 8 * kPRowBytes, kLayoutSw32);
-            tc_mma_mxf4(tmem + kColL, ad, od, idesc_mxf4(kOnesRows, 0, 0), sfp, tmem + kColSf1,
-                        j > 0 ? 1u : 0u);
+        const uint32_t sfp = tmem + kColSfP + 16 * x + 8 * pb;
+        const uint32_t sfv = tmem + kColSfV + 8 * pb;
+#pragma unroll
+        for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfp + 4 * a, sf_desc(s.psf[x][pb] + a * 512));
+        if (first) {
+#pragma unroll
+          for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfv + 4 * a, sf_desc(s.vsf[st] + a * 512));
+        }
+        const uint32_t o_col = tmem + kColO + 128 * x, l_col = tmem + kColL + 16 * x;
+        const uint32_t ones_a = smem_u32(s.ones);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 64; ++kk) {
+          const uint64_t ad = smem_desc(pa + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
+          const uint64_t bd = smem_desc(va + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
+          const uint64_t od = smem_desc(ones_a + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          if constexpr (NV) {
+            tc_mma_nvf4(o_col, ad, bd, idesc_nvf4(D), sfp + 4 * kk, sfv + 4 * kk, acc);
+            if (PNQ) tc_mma_nvf4(l_col, ad, od, idesc_nvf4(kOnesRows), sfp + 4 * kk, tmem + kColSf1, acc);
+          } else {
+            // keys 64 kk .. 64 kk + 63 are blocks 2 kk, 2 kk + 1 of the P~ and V^T scale atoms
+            tc_mma_mxf4(o_col, ad, bd, idesc_mxf4(D, 2 * kk, 2 * kk), sfp, sfv, acc);
+            if (PNQ) tc_mma_mxf4(l_col, ad, od, idesc_mxf4(kOnesRows, 2 * kk, 0), sfp, tmem + kColSf1, acc);
           }
         }
-        tc_commit(&s.bar_pv_done[j & 1]);
-        tc_commit(&s.bar_kv_empty[st]);
+        tc_commit(&s.bar_pv_done[x][pb]);
+        if (last) tc_commit(&s.bar_kv_empty[st]);
       }
       __syncwarp();
       return true;
     };
-    if (ok) ok = issue_s(0);
-    for (int j = 0; ok && j < n_kv; ++j) {
-      if (j + 1 < n_kv) ok = issue_s(j + 1);
-      if (ok) ok = issue_pv(j);
+    if (ok && n_kv_x[0] > 0) ok = issue_s(0, 0);
+    if (ok && n_kv_x[1] > 0) ok = issue_s(1, 0);
+    for (int t = 0; ok && t < n_kv_max; ++t) {
+      if (ok && t + 1 < n_kv_x[0]) ok = issue_s(0, t + 1);
+      if (ok && t < n_kv_x[0]) ok = issue_pv(0, t);
+      if (ok && t + 1 < n_kv_x[1]) ok = issue_s(1, t + 1);
+      if (ok && t < n_kv_x[1]) ok = issue_pv(1, t);
     }
     // every MMA / copy issued above must complete before TMEM is released
     if (leader) {
@@ -366,54 +403,55 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();
   } else {
-    // ============================ softmax warpgroup ============================
+    // ============================ softmax warps ============================
+    const int x = (warp - 2) >> 2;                    // query tile: warps 2-5 A, 6-9 B
     const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;                // row inside the tile == TMEM lane
+    const int qt = x == 0 ? qt_x[0] : qt_x[1];
+    const int n_kv = x == 0 ? n_kv_x[0] : n_kv_x[1];
     const int qrow = qt * kBM + r;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t o_col = tmem + lane_addr + kColO + 128 * x;
+    const uint32_t l_col = tmem + lane_addr + kColL + 16 * x;
     const float c = p.scale_log2;
+    constexpr int kPB = NV ? 16 : 32;                 // keys per P~ scale block
+    constexpr int kNPB = kBN / kPB;                   // scale blocks per row per tile
     float m = -INFINITY;      // running max of the raw scores S
     float l = 0.f;            // running row sum (pnq = 0)
-    bool ok = true;
+    bool ok = n_kv > 0;
     const bool dbg = DBG && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
-    const uint32_t p_row_off = r * kPRowBytes;
+    const uint32_t swz = (static_cast<uint32_t>(r) >> 1) & 3u;   // 64-byte swizzle of this row
     const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
-    const uint32_t swz = (static_cast<uint32_t>(r) >> 2) & 1u;   // 32-byte swizzle of this row
 
-    for (int j = 0; j < n_kv; ++j) {
-      ok = mbar_wait(&s.bar_s_full, j & 1, abort_flag, p.status, kStatusTimeoutS | 8);
-      ok = __all_sync(0xffffffffu, ok);
+    for (int t = 0; ok && t < n_kv; ++t) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8));
       if (!ok) break;
       tc_fence_after();
       float sv[kBN];
       {
-        uint32_t raw0[32], raw1[32];
-        tmem_ld32(tmem + lane_addr + kColS, raw0);
-        tmem_ld32(tmem + lane_addr + kColS + 32, raw1);
-        tc_wait_ld();
+        uint32_t raw[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = __uint_as_float(raw0[i]);
-          sv[32 + i] = __uint_as_float(raw1[i]);
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          tmem_ld32(tmem + lane_addr + kColS + 32 * cc, raw);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[32 * cc + i] = __uint_as_float(raw[i]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&s.bar_s_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.bar_s_empty);
 
       // masking: keys beyond N, and keys after the query row when causal
-      const int key0 = j * kBN;
+      const int key0 = t * kBN;
       if (key0 + kBN > p.N || (p.causal && key0 + kBN - 1 > qt * kBM)) {
+        const int lim = (p.causal ? min(p.N, qrow + 1) : p.N) - key0;   // keys [key0, key0 + lim) count
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const int key = key0 + i;
-          if (key >= p.N || (p.causal && key > qrow)) sv[i] = -INFINITY;
-        }
+        for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
       }
       // per block (32 keys for MXFP4, 16 for NVFP4): amax from the exact difference (1 for the
       // block that holds the max), the block's scale byte, and the exponent bias nb of
-      // y = P~ / s = 2^(S c - m c - log2 s): one FFMA + one ex2 per element
-      constexpr int kPB = NV ? 16 : 32;          // keys per P~ scale block
-      constexpr int kNPB = kBN / kPB;
+      // y = P~ / s = 2^(S c - m c - log2 s): one packed FMA per two elements and one ex2 each
       float bmax[kNPB];
 #pragma unroll
       for (int bb = 0; bb < kNPB; ++bb) bmax[bb] = NV ? block_max16(sv + bb * kPB) : block_max32(sv + bb * kPB);
@@ -424,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
 
-      uint32_t sbytes = 0;
+      uint32_t sbytes[kNPB / 4];
       float nb[kNPB], bscale[kNPB];
 #pragma unroll
       for (int bb = 0; bb < kNPB; ++bb) {
@@ -443,105 +481,101 @@ __global__ void __launch_bounds__(kThreads, 2)
           bscale[bb] = pow2_from_byte(byte);
           nb[bb] = fmaf(-m_use, c, static_cast<float>(127 - static_cast<int>(byte)));
         }
-        sbytes |= byte << (8 * bb);
+        if (bb % 4 == 0) sbytes[bb / 4] = 0;
+        sbytes[bb / 4] |= byte << (8 * (bb % 4));
       }
-      float y[kBN];
-#pragma unroll
-      for (int i = 0; i < kBN; ++i) y[i] = ex2_approx_ftz(fmaf(sv[i], c, nb[i / kPB]));
-      uint32_t words[kBN / 8];          // 8 words = 32 bytes of codes for this row
-#pragma unroll
-      for (int w = 0; w < kBN / 8; ++w) words[w] = cvt_e2m1x8(y + 8 * w);
-      if (!PNQ) {   // conventional row sum of the unquantized exponentials
-        float tile_sum = 0.f;
-#pragma unroll
-        for (int bb = 0; bb < kNPB; ++bb) {
-          float b0 = 0.f, b1 = 0.f;
-#pragma unroll
-          for (int i = 0; i < kPB; i += 2) {
-            b0 += y[bb * kPB + i];
-            b1 += y[bb * kPB + i + 1];
-          }
-          tile_sum = fmaf(b0 + b1, bscale[bb], tile_sum);
-        }
-        l = fmaf(alpha, l, tile_sum);
-      }
-
-      // P~ buffer j&1 is free once the product of tile j-2 (its last reader) has completed
-      const int pb = j & 1;
-      if (j >= 2) {
-        ok = mbar_wait(&s.bar_pv_done[pb], ((j >> 1) - 1) & 1, abort_flag, p.status, kStatusTimeoutPV);
-        ok = __all_sync(0xffffffffu, ok);
+      // P~ buffer t&1 is free once the product of key tile t-2 (its last reader) has completed
+      const int pb = t & 1;
+      if (t >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][pb], ((t >> 1) - 1) & 1, abort_flag, p.status,
+                                               kStatusTimeoutPV));
         if (!ok) break;
       }
-      uint8_t* p_row = s.p[pb] + p_row_off;
+      // 32 keys at a time: 16 packed FMAs, 32 ex2, four words of codes, one 16-byte store
+      uint8_t* p_row = s.p[x][pb] + r * kPRowBytes;
+      uint8_t* d_row = (DBG && dbg) ? p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) + t * kPRowBytes
+                                    : nullptr;
+      float tile_sum = 0.f;
 #pragma unroll
-      for (int bb = 0; bb < kBN / 32; ++bb) {
-        const uint4 v4 = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
-        *reinterpret_cast<uint4*>(p_row + ((bb ^ swz) << 4)) = v4;
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        float* y = sv + 32 * cc;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float x0, x1;
+          ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
+          y[i] = ex2_approx_ftz(x0);
+          y[i + 1] = ex2_approx_ftz(x1);
+        }
+        const uint4 w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
+        *reinterpret_cast<uint4*>(p_row + ((cc ^ swz) << 4)) = w4;
+        if (DBG && dbg) reinterpret_cast<uint4*>(d_row)[cc] = w4;
+        if (!PNQ) {   // conventional row sum of the unquantized exponentials
+#pragma unroll
+          for (int bb = 0; bb < 32 / kPB; ++bb) {
+            float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < kPB; i += 2) {
+              b0 += y[bb * kPB + i];
+              b1 += y[bb * kPB + i + 1];
+            }
+            tile_sum = fmaf(b0 + b1, bscale[(32 * cc) / kPB + bb], tile_sum);
+          }
+        }
       }
-      if constexpr (NV)
-        *reinterpret_cast<uint32_t*>(s.psf[pb] + psf_off) = sbytes;            // 4 blocks of 16 keys
-      else
-        *reinterpret_cast<uint16_t*>(s.psf[pb] + psf_off) = static_cast<uint16_t>(sbytes);
-      if (DBG && dbg) {
-        uint4* dc = reinterpret_cast<uint4*>(p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) +
-                                             j * kPRowBytes);
+      if (!PNQ) l = fmaf(alpha, l, tile_sum);
 #pragma unroll
-        for (int bb = 0; bb < kBN / 32; ++bb)
-          dc[bb] = make_uint4(words[bb * 4], words[bb * 4 + 1], words[bb * 4 + 2], words[bb * 4 + 3]);
-        if constexpr (NV)
-          *reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 16) + j * 4) =
-              sbytes;
-        else
-          *reinterpret_cast<uint16_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 32) + j * 2) =
-              static_cast<uint16_t>(sbytes);
+      for (int a = 0; a < kNPB / 4; ++a) *reinterpret_cast<uint32_t*>(s.psf[x][pb] + a * 512 + psf_off) = sbytes[a];
+      if (DBG && dbg) {
+        uint32_t* ds = reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) *
+                                                                      (p.Npad / kPB) + t * kNPB);
+#pragma unroll
+        for (int a = 0; a < kNPB / 4; ++a) ds[a] = sbytes[a];
       }
       fence_proxy_async_smem();
 
       // history rescale of O and L (only when some row of this warp saw its max move); O may only
-      // be touched once the product of tile j-1 has landed in it
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        ok = mbar_wait(&s.bar_pv_done[pb ^ 1], ((j - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
-        ok = __all_sync(0xffffffffu, ok);
+      // be touched once the product of key tile t-1 has landed in it
+      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag,
+                                               p.status, kStatusTimeoutPV | 4));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; cc += 2) {   // 64 columns per round trip
-          uint32_t raw0[32], raw1[32];
-          const uint32_t col = tmem + lane_addr + kColO + cc * 32;
-          tmem_ld32(col, raw0);
-          tmem_ld32(col + 32, raw1);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t raw[32];
+          tmem_ld32(o_col + cc * 32, raw);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            raw0[i] = __float_as_uint(__uint_as_float(raw0[i]) * alpha);
-            raw1[i] = __float_as_uint(__uint_as_float(raw1[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            float o0, o1;
+            fmul2_b(o0, o1, __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]), alpha);
+            raw[i] = __float_as_uint(o0);
+            raw[i + 1] = __float_as_uint(o1);
           }
-          tmem_st32(col, raw0);
-          tmem_st32(col + 32, raw1);
+          tmem_st32(o_col + cc * 32, raw);
         }
         if (PNQ) {
-          const uint32_t lv = tmem_ld1(tmem + lane_addr + kColL);
+          const uint32_t lv = tmem_ld1(l_col);
           tc_wait_ld();
-          tmem_st1(tmem + lane_addr + kColL, __float_as_uint(__uint_as_float(lv) * alpha));
+          tmem_st1(l_col, __float_as_uint(__uint_as_float(lv) * alpha));
         }
         tc_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&s.bar_p_full[pb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.bar_p_full[x][pb]);
       m = m_new;
     }
 
     // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
     if (ok) {
-      ok = mbar_wait(&s.bar_pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
-                     kStatusTimeoutPV | 1);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag,
+                                             p.status, kStatusTimeoutPV | 1));
     }
     if (ok) {
       tc_fence_after();
       if (PNQ) {
-        l = __uint_as_float(tmem_ld1(tmem + lane_addr + kColL));
+        l = __uint_as_float(tmem_ld1(l_col));
         tc_wait_ld();
       }
       const float inv_l = 1.f / l;
@@ -550,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_addr + kColO + cc * 32, raw);
+        tmem_ld32(o_col + cc * 32, raw);
         tc_wait_ld();
         if (store) {
           if (p.out_bf16) {
@@ -559,10 +593,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int v = 0; v < 4; ++v) {
               uint32_t wv[4];
 #pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * t]) * inv_l,
-                                                                __uint_as_float(raw[v * 8 + 2 * t + 1]) * inv_l);
-                wv[t] = *reinterpret_cast<const uint32_t*>(&h2);
+              for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * u]) * inv_l,
+                                                                __uint_as_float(raw[v * 8 + 2 * u + 1]) * inv_l);
+                wv[u] = *reinterpret_cast<const uint32_t*>(&h2);
               }
               dst[v] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
@@ -594,7 +628,8 @@ static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
   cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ, DBG, NV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * (p.Npad / kBM);
+  const unsigned n_units = static_cast<unsigned>((p.Npad / kBM + 1) / 2);
+  const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * n_units;
   mxattn_fwd_kernel<D, PNQ, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }

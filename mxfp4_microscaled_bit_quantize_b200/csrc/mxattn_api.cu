@@ -197,7 +197,7 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   if (!make_map(&tq, src.qc, d / 2, static_cast<uint64_t>(B) * Hq * rph, d / 2, kTile, qk_swz) ||
       !make_map(&tk, src.kc, d / 2, static_cast<uint64_t>(B) * Hkv * rph, d / 2, kKvTile, qk_swz) ||
       !make_map(&tv, src.vc, src.v_row_bytes, static_cast<uint64_t>(B) * Hkv * d, kKvTile / 2, d,
-                CU_TENSOR_MAP_SWIZZLE_32B))
+                CU_TENSOR_MAP_SWIZZLE_64B))
     return MXATTN_ERR_CUDA;
   AttnParams p{};
   p.qsf = w + L.qs;

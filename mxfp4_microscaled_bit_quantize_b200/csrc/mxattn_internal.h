@@ -9,7 +9,7 @@ namespace mxattn {
 
 // Keys per KV tile of the attention kernel: P~ is quantized with the running max in force at
 // each tile, so this width is part of what the kernel computes (MXATTN_KV_TILE in mxattn.h).
-constexpr int kKvTile = 64;
+constexpr int kKvTile = 128;
 
 enum SfLayout : int { kSfRowMajor = 0, kSfAtom = 1 };
 

@@ -277,6 +277,50 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t n, uint32_t a_sf_id, 
          (a_sf_id << 29);
 }
 
+// Two fp32 FMAs in one packed instruction (sm_100+): (a0, a1) * b + (c, c).
+__device__ __forceinline__ void ffma2_bc(float& r0, float& r1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// Two fp32 products in one packed instruction: (a0, a1) * (b, b).
+__device__ __forceinline__ void fmul2_b(float& r0, float& r1, float a0, float a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b));
+}
+
+// Named barrier ID (an immediate, so that the kernel reserves only the barriers it names) over
+// COUNT threads (whole warps), returning the AND of `v` over them.
+template <int ID, int COUNT>
+__device__ __forceinline__ bool bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(ID), "n"(COUNT)
+      : "memory");
+  return r != 0;
+}
+
+template <int ID, int COUNT>
+__device__ __forceinline__ void bar_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(COUNT) : "memory");
+}
+
 // max(a, b, c) in one instruction (three-input form, sm_100+).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

@@ -53,7 +53,7 @@ import numpy as np
 from . import mxfp4 as mx
 from . import nvfp4 as nv
 
-KV_TILE = 64          # the library's documented tile width (MXATTN_KV_TILE)
+KV_TILE = 128         # the library's documented tile width (MXATTN_KV_TILE)
 
 
 def dequantized_qkv(q, k, v, mode: int):
