@@ -300,10 +300,11 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         torch.cuda.synchronize(dev)
 
     mode = {"uos": api.SCALE_UOS, "ocp": api.SCALE_OCP, "nvfp4": api.SCALE_NVFP4}[args.scale]
+    p_rule = {"conventional": api.P_CONVENTIONAL, "pnq": api.P_PNQ, "efq": api.P_EFQ}[args.p_rule]
 
     def step():
         api.mxattn_forward_prepare(dq, dk, dv, mode, ws)
-        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, True, ws)
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, p_rule, ws)
 
     for _ in range(args.warmup):
         step()
@@ -319,7 +320,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             ev[i][0].record(stream)
             api.mxattn_forward_prepare(dq, dk, dv, mode, ws)
             ev[i][1].record(stream)
-            api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, True, ws)
+            api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, mode, p_rule, ws)
             ev[i][2].record(stream)
         stop.record(stream)
         barrier()
@@ -329,7 +330,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     quant_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
     if args.mode == "attention":
-        print(json.dumps({"mode": "attention", "scale": args.scale, "config": cfg.describe(), "attn_ms": attn_ms,
+        print(json.dumps({"mode": "attention", "scale": args.scale, "p_rule": args.p_rule, "config": cfg.describe(),
+                          "attn_ms": attn_ms,
                           "quant_ms": quant_ms, "tflops": cfg.flops / (attn_ms * 1e-3) / 1e12}), flush=True)
         return
 
@@ -417,6 +419,20 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         raise RuntimeError("device pipeline timeout in the NVFP4 attention")
     nv_attn_ms = n_start.elapsed_time(n_stop) / fq_steps
 
+    # the exp-free P~ rule (EFQ-Softmax reading) in the same kernel, UOS scales, attention alone
+    api.mxattn_forward_prepare(dq, dk, dv, api.SCALE_UOS, ws)
+    for _ in range(2):
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, api.P_EFQ, ws)
+    barrier()
+    n_start.record(stream)
+    for _ in range(fq_steps):
+        api.mxattn_forward_attend(out, B, Hq, Hkv, N, d, cfg.causal, api.SCALE_UOS, api.P_EFQ, ws)
+    n_stop.record(stream)
+    barrier()
+    if api.mxattn_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout in the exp-free attention")
+    efq_attn_ms = n_start.elapsed_time(n_stop) / fq_steps
+
     # the other full-size attention workloads: the long video DiT and the causal GQA prefill
     # (quantizers + attention kernel per step, timed per phase as in the main loop)
     other = {}
@@ -490,8 +506,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     # max over ranks
     other_ms = [x for name in OTHER_CONFIGS for x in other[name][1:]]
     (step_ms, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
-     nv_attn_ms, *other_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms, copy_ms,
-                                                     quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms,
+     nv_attn_ms, efq_attn_ms, *other_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms,
+                                                     copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms,
+                                                     efq_attn_ms,
                                                      *other_ms], world, dev)
     if rank != 0:
         return
@@ -533,6 +550,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                                             f"{QUANT_SETS * qa_bytes / 1e6:.0f} MB in all (> 2 x 126 MB L2)",
                       "standalone_frac": qa_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "traffic": profile_traffic("quantize_rows_65536x1024.json", sources_hash(QUANT_SOURCES))},
+        "exp_free_attention": {"ms": efq_attn_ms, "tflops": flops / (efq_attn_ms * 1e-3) / 1e12,
+                               "frac": flops / (efq_attn_ms * 1e-3) / 1e12 / fp4_peak,
+                               "note": "pnq = MXATTN_P_EFQ (exp-free P~ codes, EFQ-Softmax reading), UOS, "
+                                       "attention kernel alone; a different P~ rule from the headline"},
         "nvfp4_attention": {"ms": nv_attn_ms, "tflops": flops / (nv_attn_ms * 1e-3) / 1e12,
                             "note": "MXATTN_SCALE_NVFP4 (Q, K, V, P~ in NVFP4), attention kernel alone",
                             "traffic": profile_traffic("attn_fwd_video_dit_nvfp4.json", sources_hash(ATTN_SOURCES))},
@@ -643,11 +664,15 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
     ap.add_argument("--workload", choices=[WORKLOAD, *OTHER_CONFIGS], default=WORKLOAD,
                     help="the attention workload of --mode attention (profiling only)")
+    ap.add_argument("--p-rule", choices=["conventional", "pnq", "efq"], default="pnq",
+                    help="the P~ rule of --mode attention (profiling only)")
     ap.add_argument("--scale", choices=["uos", "ocp", "nvfp4"], default="uos",
                     help="the scale mode of --mode attention (profiling only)")
     args = ap.parse_args()
     if args.workload != WORKLOAD and (args.mode != "attention" or args.heads):
         ap.error("--workload applies to --mode attention, without --heads")
+    if args.p_rule != "pnq" and args.mode != "attention":
+        ap.error("--p-rule applies to --mode attention")
     if args.scale != "uos" and args.mode != "attention":
         ap.error("--scale applies to --mode attention")
     if args.warmup < 3:

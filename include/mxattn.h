@@ -24,6 +24,13 @@
  *     the unnormalised exponentials P~ = exp(S/sqrt(d) - m) are quantized to MXFP4 along keys
  *     before the row sum, and that same dequantized operand feeds both P~V and the row sum.
  *     With pnq = 0 the row sum uses the unquantized fp32 P~ (exp-then-quantize baseline).
+ *     With pnq = 2 the P~ operand is made without exponentials, after the EFQ-Softmax abstract:
+ *     per 32-key block the scale exponent e is the block's MXFP4 exponent (OCP or UOS) of its
+ *     largest P~, and each key gets the code k = clamp(round_half_even(2 r + 2), 0, 7) of its
+ *     residual r = log2(P~) - e; that operand feeds both P~V and the row sum, as under PNQ.
+ *     (The abstract gives the structure -- exponent-only scale from the block max, residual
+ *     domain, one affine rule -- but no constants; 2 r + 2 is the reading that lands on the
+ *     grid values 1, 2 and 4 at r = 0, 1, 2.) MXFP4 scale modes only.
  *     Softmax scale is fixed at 1/sqrt(d).
  *
  * Conventions
@@ -58,6 +65,12 @@ typedef enum { MXATTN_SCALE_OCP = 0, MXATTN_SCALE_UOS = 1, MXATTN_SCALE_NVFP4 = 
 /* Keys per tile of the online softmax. P~ is quantized with the running max in force at each
  * tile, so the tile width is part of the result (a CPU reference must use the same width). */
 #define MXATTN_KV_TILE 128
+
+/* Values of the `pnq` argument of the attention entry points: the rule that makes the P~ operand
+ * and its row sum (see "What it computes" above). */
+#define MXATTN_P_CONVENTIONAL 0   /* exp-then-quantize, row sum of the unquantized P~ */
+#define MXATTN_P_PNQ 1            /* exp-then-quantize, row sum of the same quantized operand */
+#define MXATTN_P_EFQ 2            /* exp-free codes, row sum of the same operand (MXFP4 only) */
 
 typedef enum { MXATTN_OUT_F32 = 0, MXATTN_OUT_BF16 = 1 } mxattn_out_dtype;
 
@@ -100,6 +113,8 @@ size_t mxattn_forward_workspace_size(int B, int Hq, int Hkv, int N, int d);
  *   out : [B, Hq, N, d] fp32 (out_dtype = MXATTN_OUT_F32) or bf16, device, 16-byte aligned
  *   Query head h reads KV head h / (Hq / Hkv) (contiguous GQA groups); Hq % Hkv == 0.
  *   causal = 1 masks keys after the query position. scale_mode applies to Q, K, V and P~.
+ *   pnq: MXATTN_P_CONVENTIONAL, MXATTN_P_PNQ or MXATTN_P_EFQ (any other value ->
+ *   MXATTN_ERR_INVALID_ARG; MXATTN_P_EFQ with MXATTN_SCALE_NVFP4 -> MXATTN_ERR_UNSUPPORTED).
  *   Supported: d in {64, 128}, 1 <= N, B*Hq*ceil(N/128) < 2^31.
  *   workspace: device memory of at least mxattn_forward_workspace_size(...) bytes, 256-byte
  *   aligned; its contents on entry are ignored; it must not be used concurrently by another
@@ -111,7 +126,7 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* 
 
 /*
  * mxattn_forward_quantized -- the attention kernel alone, on Q, K and V already in MXFP4 (MXAttention
- * abstract: MXFP4 operands for Q K^T and P~ V; P~ is quantized inside, with PNQ when pnq = 1).
+ * abstract: MXFP4 operands for Q K^T and P~ V; P~ is quantized inside by the rule `pnq` names).
  * The operands are in the canonical layout that mxattn_quantize writes:
  *   qc  : codes  [B, Hq,  N, d/2]   (mxattn_quantize of q, transpose = 0), 16-byte aligned
  *   qs  : scales [B, Hq,  N, d/32]  E8M0 bytes

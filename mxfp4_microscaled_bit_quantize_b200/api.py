@@ -11,6 +11,7 @@ import torch
 from . import _lib
 
 SCALE_OCP, SCALE_UOS, SCALE_NVFP4 = 0, 1, 2
+P_CONVENTIONAL, P_PNQ, P_EFQ = 0, 1, 2   # the `pnq` argument (MXATTN_P_*): rule of the P~ operand
 OUT_F32, OUT_BF16 = 0, 1
 KV_TILE = 128         # keys per online-softmax tile (MXATTN_KV_TILE)
 NPAD_ALIGN = 128      # the workspace pads N to a multiple of this
@@ -105,7 +106,7 @@ def mxattn_forward(q, k, v, causal: bool = False, scale_mode: int = SCALE_UOS, p
         workspace = alloc_workspace(B, Hq, Hkv, N, d, q.device)
     lib = _lib.load()
     st = lib.mxattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
-                            int(bool(causal)), int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                            int(bool(causal)), int(scale_mode), int(pnq), od, workspace.data_ptr(),
                             workspace.numel(), _stream(q.device))
     _lib.check(st, "mxattn_forward")
     return out
@@ -134,7 +135,7 @@ def mxattn_forward_host(q, k, v, out, causal: bool = False, scale_mode: int = SC
             raise ValueError("unsupported attention shape")
         workspace = torch.empty(n, dtype=torch.uint8, device=dev)
     st = lib.mxattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
-                                 int(bool(causal)), int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                                 int(bool(causal)), int(scale_mode), int(pnq), od, workspace.data_ptr(),
                                  workspace.numel(), _stream(dev))
     _lib.check(st, "mxattn_forward_host")
     return out
@@ -166,7 +167,7 @@ def mxattn_forward_quantized(qc, qs, kc, ks, vtc, vts, N: int, d: int, causal: b
         workspace = alloc_workspace(B, Hq, Hkv, N, d, qc.device)
     st = _lib.load().mxattn_forward_quantized(qc.data_ptr(), qs.data_ptr(), kc.data_ptr(), ks.data_ptr(),
                                               vtc.data_ptr(), vts.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
-                                              int(bool(causal)), int(p_scale_mode), int(bool(pnq)), od,
+                                              int(bool(causal)), int(p_scale_mode), int(pnq), od,
                                               workspace.data_ptr(), workspace.numel(), _stream(qc.device))
     _lib.check(st, "mxattn_forward_quantized")
     return out
@@ -259,7 +260,7 @@ def mxattn_forward_attend(out: torch.Tensor, B: int, Hq: int, Hkv: int, N: int, 
                           scale_mode: int, pnq: bool, workspace: torch.Tensor) -> torch.Tensor:
     od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     st = _lib.load().mxattn_forward_attend(out.data_ptr(), B, Hq, Hkv, N, d, int(bool(causal)),
-                                           int(scale_mode), int(bool(pnq)), od, workspace.data_ptr(),
+                                           int(scale_mode), int(pnq), od, workspace.data_ptr(),
                                            workspace.numel(), _stream(out.device))
     _lib.check(st, "mxattn_forward_attend")
     return out
@@ -278,7 +279,7 @@ def mxattn_forward_debug(q, k, v, dbg_bh: int, r0: int, r1: int, causal: bool = 
     pc = torch.zeros((r1 - r0, npd // 2), dtype=torch.uint8, device=q.device)
     ps = torch.zeros((r1 - r0, npd // (16 if scale_mode == SCALE_NVFP4 else 32)), dtype=torch.uint8, device=q.device)
     st = _lib.load().mxattn_forward_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
-                                          Hkv, N, d, int(bool(causal)), int(scale_mode), int(bool(pnq)), od,
+                                          Hkv, N, d, int(bool(causal)), int(scale_mode), int(pnq), od,
                                           workspace.data_ptr(), workspace.numel(), _stream(q.device),
                                           dbg_bh, r0, r1, pc.data_ptr(), ps.data_ptr())
     _lib.check(st, "mxattn_forward_debug")

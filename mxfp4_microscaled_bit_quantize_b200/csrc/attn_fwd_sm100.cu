@@ -21,14 +21,16 @@
 // S(A, t+1), ... . Their softmax warps therefore run half a step apart, and on every SM
 // sub-partition one tile's serial work (S load, maxima, scale selection, stores, rescale) overlaps
 // the other tile's exponentials on the MUFU.
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 72 registers
+// per thread and each softmax warpgroup 216):
 //   warp 0     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
 //              an NSTAGE-deep shared-memory ring (mbarrier complete_tx).
+//   warps 2, 3 no role (they complete the control warpgroup).
 //   warp 1     TMEM owner and MMA issuer (one thread): copies scale atoms to TMEM with tcgen05.cp
 //              and issues, per key tile t, S(A, t+1), O_A += P~_A(t) V(t) (+ L_A), S(B, t+1),
 //              O_B += P~_B(t) V(t) (+ L_B). Each S waits until the previous user of the S buffer
 //              holds its scores in registers.
-//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one thread per query row (TMEM lane = row).
+//   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per query row (TMEM lane = row).
 //              Per key tile a thread reads its 128 scores with tcgen05.ld, releases S, updates the
 //              running max, computes P~ / 2^e per 32-key block, quantizes it in registers, writes
 //              64 bytes of codes (64B-swizzled, the MMA operand layout) and four scale bytes to
@@ -38,7 +40,13 @@
 // scale atoms from 416 (see kColSf*).
 // The kernel is templated on the format: MXFP4 (the method) or, for comparison, NVFP4 (blocks of
 // 16 with E4M3 scales for Q, K, V and P~; kind::mxf4nvf4 products, the non-power-of-two P~ scale
-// folded into the exponent bias as -log2 s).
+// folded into the exponent bias as -log2 s), and on the rule that makes the P~ operand:
+//   PM = 0  exp-then-quantize, row sum of the unquantized exponentials (the conventional path)
+//   PM = 1  exp-then-quantize, row sum of the same quantized operand (PNQ)
+//   PM = 2  exp-free codes (EFQ-Softmax abstract): per 32-key block the exponent-only scale of
+//           the block max as above, then code k = clamp(round(2 r + 2), 0, 7) of the residual
+//           r = S c - m c - e (the base-2 log of P~ / 2^e), no exponential per element; the row
+//           sum again comes from the same operand. MXFP4 only.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -50,8 +58,12 @@ namespace mxattn {
 
 constexpr int kBM = 128;          // query rows per Q tile (the MMA's M)
 constexpr int kBN = kKvTile;      // keys per KV tile (128)
-constexpr int kSoftmaxWarps = 8;  // four per query tile
-constexpr int kThreads = 64 + 32 * kSoftmaxWarps;   // 320: producer, MMA, softmax A, softmax B
+constexpr int kThreads = 384;     // warpgroup 0: producer, MMA, 2 idle; warpgroups 1, 2: softmax A, B
+// Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for 384
+// threads); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to kSoftmaxRegs.
+// The three shares add up to exactly the launch total, which the host checks before launching.
+constexpr int kLaunchRegs = 168, kCtlRegs = 72, kSoftmaxRegs = 216;
+static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 X, L_X at kColL + 16 X
 // Scale atoms, 4 columns each (NVFP4 needs two per operand tile, MXFP4 one):
@@ -123,6 +135,58 @@ __device__ __forceinline__ float ex2_approx_ftz(float x) {
   return y;
 }
 
+// 2^x on the FMA and ALU pipes, for a share of the PNQ exponentials that would otherwise queue on
+// the MUFU. Only the E2M1 code of 2^x is kept, so the function has to fall on the correct side of
+// every rounding midpoint of the grid (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 times 2^e), not be
+// accurate everywhere. Range reduction x = n + f with n = round(x), f in [-0.5, 0.5] (the
+// 1.5 * 2^23 bias rounds to an integer in the mantissa); 2^f by the cubic through 2^f at
+// f = log2 0.75, log2 0.875 and log2 1.25, with value 1 at f = 0 -- the four places where a
+// midpoint of the grid falls after the reduction (log2 1.75 - 1 = log2 0.875). Between them the
+// cubic is within 4e-4 of 2^f and increasing, which no code can see; at them it is within one
+// fp32 ulp, like ex2.approx. The coefficients were fitted in fp64 and rounded to fp32. x is
+// clamped at -127 so that n << 23 stays inside the exponent field (such values code to 0
+// anyway).
+__device__ __forceinline__ void exp2_codes_poly(float& y0, float& y1, float x0, float x1) {
+  constexpr float kRound = 12582912.0f;                       // 1.5 * 2^23
+  constexpr float kC1 = 0x1.630374p-1f, kC2 = 0x1.ee3f4ep-3f, kC3 = 0x1.b240f2p-5f;
+  const float xc0 = fmaxf(x0, -127.f), xc1 = fmaxf(x1, -127.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0, t1, xc0, xc1, kRound, kRound);
+  fadd2(n0, n1, t0, t1, -kRound, -kRound);
+  fadd2(f0, f1, xc0, xc1, -n0, -n1);
+  ffma2(p0, p1, f0, f1, kC3, kC3, kC2, kC2);
+  ffma2(p0, p1, p0, p1, f0, f1, kC1, kC1);
+  ffma2(p0, p1, p0, p1, f0, f1, 1.f, 1.f);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// Wait of a whole warp for an mbarrier phase (bounded, see mbar_wait). kSpin polls instead of
+// suspending: the MMA issuer uses it under the exp-free rule, where the softmax phase is short and
+// the S-buffer hand-over (softmax release -> MMA issue -> next softmax) sets the pace.
+template <bool kSpin = false>
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* status, unsigned int code) {
+  if constexpr (kSpin) return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, status, code));
+  else return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, code));
+}
+
+// E8M0 byte of a P~ block maximum amax in [0, 1] (the running max bounds every P~ by 1): the OCP
+// exponent floor(log2 amax) - 2 read off the fp32 exponent field, plus one under UOS when the
+// significand exceeds 1.8125; byte 0 for amax = 0 and for every amax whose exponent would fall
+// below -127 (subnormal or tiny maxima), as the general rule's clamp gives.
+__device__ __forceinline__ uint32_t p_scale_byte(float amax, int mode) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int byte = static_cast<int>(bits >> 23) - 2 + ((mode == 1 && (bits & 0x7FFFFFu) > 0x680000u) ? 1 : 0);
+  return static_cast<uint32_t>(max(byte, 0));
+}
+
+// Every kPolyEvery-th pair of keys takes its PNQ exponentials from exp2_codes_poly instead of the
+// MUFU (0: all on the MUFU). Measured on the video-DiT workload with 1/8, 1/4 and 1/2 of the
+// exponentials moved: no gain, because the MUFU is not what bounds the kernel (the exp-free rule,
+// which needs no exponential at all, runs only about a fifth faster); kept off.
+constexpr int kPolyEvery = 0;
+
 // Bounded wait that ignores the abort flag (used only to drain in-flight copies / MMAs).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
@@ -164,10 +228,13 @@ __device__ __forceinline__ float lg2_approx(float x) {
 
 // NV = false: MXFP4 (blocks of 32, UE8M0, OCP or UOS exponent). NV = true: the NVFP4 comparison
 // format for Q, K, V and P~ (blocks of 16, E4M3 scale = RNE(amax / 6)).
-template <int D, bool PNQ, bool DBG, bool NV>
+template <int D, int PM, bool DBG, bool NV>
 __global__ void __launch_bounds__(kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  static_assert(PM >= 0 && PM <= 2 && !(NV && PM == 2), "P~ rule");
+  constexpr bool PNQ = PM != 0;     // the row sum is the ones-operand product of the quantized P~
+  constexpr bool EFQ = PM == 2;
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
   constexpr int kQKAtoms = NV ? D / 64 : 1;            // scale atoms per 128 Q or K rows
@@ -231,7 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<kCtlRegs>();
+   if (warp == 0) {
     // ============================ TMA producer ============================
     // The whole warp runs the loop (warp-uniform operands); one elected lane issues the copies.
     const bool leader = elect_one_sync();
@@ -251,9 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < n_kv_max; ++t) {
       const int st = t % NS;
       if (t >= NS) {
-        bool ok = mbar_wait(&s.bar_kv_empty[st], ((t / NS) & 1) ^ 1, abort_flag, p.status,
-                            kStatusTimeoutEmpty | st);
-        if (!__all_sync(0xffffffffu, ok)) break;
+        if (!warp_wait(&s.bar_kv_empty[st], ((t / NS) & 1) ^ 1, abort_flag, p.status, kStatusTimeoutEmpty | st))
+          break;
       }
       if (leader) {
         mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + kQKSfBytes + kPVSfBytes);
@@ -300,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     const bool leader = elect_one_sync();
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_q, 0, abort_flag, p.status, kStatusTimeoutQ));
+    bool ok = warp_wait(&s.bar_q, 0, abort_flag, p.status, kStatusTimeoutQ);
     if (ok) {
       tc_fence_after();
       if (leader) {
@@ -312,29 +380,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    // Shared-memory descriptors: only the 14-bit start-address field (16-byte units) differs between
+    // the operands of one kind, so each is one OR of a fixed upper part with an address.
+    const uint64_t d_qk = smem_desc(0, 0, C::kQKSbo, C::kQKLayout);          // Q and K tiles
+    const uint64_t d_pv = smem_desc(0, 0, 8 * kPRowBytes, kLayoutSw64);      // P~, V^T and ones tiles
+    const uint32_t a_q = smem_u32(s.q[0]) >> 4, a_k = smem_u32(s.k[0]) >> 4, a_v = smem_u32(s.v[0]) >> 4;
+    const uint32_t a_p = smem_u32(s.p[0][0]) >> 4, a_ones = smem_u32(s.ones) >> 4;
     int s_uses = 0;      // S products issued so far (A and B alternate on the one buffer)
     auto issue_s = [&](int x, int t) -> bool {
       const int st = t % NS;
       const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
-      if (first && !__all_sync(0xffffffffu, mbar_wait(&s.bar_kv_full[st], (t / NS) & 1, abort_flag, p.status,
-                                                       kStatusTimeoutKV | st)))
-        return false;
-      // the previous user of the S buffer must hold its scores in registers
-      if (s_uses > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status,
-                                                           kStatusTimeoutS)))
-        return false;
-      tc_fence_after();
-      const uint32_t qa = smem_u32(s.q[x]), ka = smem_u32(s.k[st]);
       const uint32_t sfk = tmem + kColSfK + 8 * (t & 1);
-      if (leader) {
-        if (first) {
+      if (first) {
+        if (!warp_wait<EFQ>(&s.bar_kv_full[st], (t / NS) & 1, abort_flag, p.status,
+                                            kStatusTimeoutKV | st))
+          return false;
+        // the K atoms of tile t go to the set the S products of tile t - 2 read; those completed
+        // before the S buffer's user of S(t - 1) could read it, which this thread waited for when it
+        // issued the S product that followed (or there was none)
+        tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(sfk + 4 * a, sf_desc(s.ksf[st] + a * 512));
         }
+      }
+      // the previous user of the S buffer must hold its scores in registers
+      if (s_uses > 0 &&
+          !warp_wait<EFQ>(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
+        return false;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t qa = a_q + x * (C::kQTileBytes >> 4), ka = a_k + st * (C::kKTileBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk) {
-          const uint64_t ad = smem_desc(qa + kk * 32, 0, C::kQKSbo, C::kQKLayout);
-          const uint64_t bd = smem_desc(ka + kk * 32, 0, C::kQKSbo, C::kQKLayout);
+          const uint64_t ad = d_qk | (qa + kk * 2), bd = d_qk | (ka + kk * 2);   // +32 bytes per K = 64
           if constexpr (NV)   // one atom (four 16-element blocks) per K = 64 step
             tc_mma_nvf4(tmem + kColS, ad, bd, idesc_nvf4(kBN), tmem + kColSfQ + 8 * x + 4 * kk, sfk + 4 * kk, kk > 0);
           else
@@ -349,13 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](int x, int t) -> bool {
       const int st = t % NS;
       const int pb = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status,
-                                             kStatusTimeoutP)))
+      if (!warp_wait<EFQ>(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status, kStatusTimeoutP))
         return false;
       tc_fence_after();
       const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
       const bool last = (x == 1) || t >= n_kv_x[1];       // last reader of the tile's stage
-      const uint32_t pa = smem_u32(s.p[x][pb]), va = smem_u32(s.v[st]);
       if (leader) {
         const uint32_t sfp = tmem + kColSfP + 16 * x + 8 * pb;
         const uint32_t sfv = tmem + kColSfV + 8 * pb;
@@ -366,12 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfv + 4 * a, sf_desc(s.vsf[st] + a * 512));
         }
         const uint32_t o_col = tmem + kColO + 128 * x, l_col = tmem + kColL + 16 * x;
-        const uint32_t ones_a = smem_u32(s.ones);
+        const uint32_t pa = a_p + (2 * x + pb) * ((kBM * kPRowBytes) >> 4), va = a_v + st * (C::kVTileBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 64; ++kk) {
-          const uint64_t ad = smem_desc(pa + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
-          const uint64_t bd = smem_desc(va + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
-          const uint64_t od = smem_desc(ones_a + kk * 32, 0, 8 * kPRowBytes, kLayoutSw64);
+          const uint64_t ad = d_pv | (pa + kk * 2), bd = d_pv | (va + kk * 2), od = d_pv | (a_ones + kk * 2);
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
           if constexpr (NV) {
             tc_mma_nvf4(o_col, ad, bd, idesc_nvf4(D), sfp + 4 * kk, sfv + 4 * kk, acc);
@@ -402,9 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&s.bar_drain, 0);
     }
     __syncwarp();
+   }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ============================ softmax warps ============================
-    const int x = (warp - 2) >> 2;                    // query tile: warps 2-5 A, 6-9 B
+    const int x = (warp - 4) >> 2;                    // query tile: warps 4-7 A, 8-11 B
     const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;                // row inside the tile == TMEM lane
     const int qt = x == 0 ? qt_x[0] : qt_x[1];
@@ -416,6 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     constexpr int kPB = NV ? 16 : 32;                 // keys per P~ scale block
     constexpr int kNPB = kBN / kPB;                   // scale blocks per row per tile
+    const float c27 = c * (2.f / 7.f);                // exp-free rule: (2 r + 2) / 7 = S c27 + b7
     float m = -INFINITY;      // running max of the raw scores S
     float l = 0.f;            // running row sum (pnq = 0)
     bool ok = n_kv > 0;
@@ -424,19 +502,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
 
     for (int t = 0; ok && t < n_kv; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8));
+      ok = warp_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8);
       if (!ok) break;
       tc_fence_after();
       float sv[kBN];
       {
-        uint32_t raw[32];
+        uint32_t raw[kBN];
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          tmem_ld32(tmem + lane_addr + kColS + 32 * cc, raw);
-          tc_wait_ld();
+        for (int cc = 0; cc < kBN / 32; ++cc)
+          tmem_ld32(tmem + lane_addr + kColS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
+        tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[32 * cc + i] = __uint_as_float(raw[i]);
-        }
+        for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(raw[i]);
       }
       tc_fence_before();
       __syncwarp();
@@ -477,9 +554,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           bscale[bb] = sb > 0.f ? sb : 1.f;
           nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
         } else {
-          byte = e8m0_scale_byte(amax, p.mode);
+          byte = p_scale_byte(amax, p.mode);
+          // 127 - byte as a float without a conversion: it sits in the low mantissa bits of 2^23
+          const float neg_e = __uint_as_float(0x4B000000u + (127u - byte)) - 8388608.0f;
+          nb[bb] = fmaf(-m_use, c, neg_e);
           bscale[bb] = pow2_from_byte(byte);
-          nb[bb] = fmaf(-m_use, c, static_cast<float>(127 - static_cast<int>(byte)));
         }
         if (bb % 4 == 0) sbytes[bb / 4] = 0;
         sbytes[bb / 4] |= byte << (8 * (bb % 4));
@@ -487,8 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P~ buffer t&1 is free once the product of key tile t-2 (its last reader) has completed
       const int pb = t & 1;
       if (t >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][pb], ((t >> 1) - 1) & 1, abort_flag, p.status,
-                                               kStatusTimeoutPV));
+        ok = warp_wait(&s.bar_pv_done[x][pb], ((t >> 1) - 1) & 1, abort_flag, p.status, kStatusTimeoutPV);
         if (!ok) break;
       }
       // 32 keys at a time: 16 packed FMAs, 32 ex2, four words of codes, one 16-byte store
@@ -499,14 +577,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < kBN / 32; ++cc) {
         float* y = sv + 32 * cc;
+        uint4 w4;
+        if constexpr (EFQ) {
+          // w = sat((2 r + 2) / 7); w times 7 * 2^-149 lands on the subnormal grid, so the product's
+          // bit pattern is round(7 w) in [0, 7] (round to nearest even): the code itself
+          const float b7 = fmaf(nb[cc], 2.f / 7.f, 2.f / 7.f);
+          uint32_t wd[4];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float x0, x1;
-          ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
-          y[i] = ex2_approx_ftz(x0);
-          y[i + 1] = ex2_approx_ftz(x1);
+          for (int w = 0; w < 4; ++w) {
+            float k[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) k[i] = fma_sat(y[8 * w + i], c27, b7);
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) fmul2_b(k[i], k[i + 1], k[i], k[i + 1], __uint_as_float(7u));
+            uint32_t acc = pack_u4x2(0u, __float_as_uint(k[7]), __float_as_uint(k[6]));
+            acc = pack_u4x2(acc, __float_as_uint(k[5]), __float_as_uint(k[4]));
+            acc = pack_u4x2(acc, __float_as_uint(k[3]), __float_as_uint(k[2]));
+            wd[w] = pack_u4x2(acc, __float_as_uint(k[1]), __float_as_uint(k[0]));
+          }
+          w4 = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
+            if (PM == 1 && !NV && kPolyEvery > 0 && (i / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+              exp2_codes_poly(y[i], y[i + 1], x0, x1);
+            } else {
+              y[i] = ex2_approx_ftz(x0);
+              y[i + 1] = ex2_approx_ftz(x1);
+            }
+          }
+          w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
         }
-        const uint4 w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
         *reinterpret_cast<uint4*>(p_row + ((cc ^ swz) << 4)) = w4;
         if (DBG && dbg) reinterpret_cast<uint4*>(d_row)[cc] = w4;
         if (!PNQ) {   // conventional row sum of the unquantized exponentials
@@ -536,23 +639,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // history rescale of O and L (only when some row of this warp saw its max move); O may only
       // be touched once the product of key tile t-1 has landed in it
       if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag,
-                                               p.status, kStatusTimeoutPV | 4));
+        ok = warp_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t raw[32];
-          tmem_ld32(o_col + cc * 32, raw);
+        {
+          uint32_t raw[D];
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc)
+            tmem_ld32(o_col + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
+          for (int i = 0; i < D; i += 2) {
             float o0, o1;
             fmul2_b(o0, o1, __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]), alpha);
             raw[i] = __float_as_uint(o0);
             raw[i + 1] = __float_as_uint(o1);
           }
-          tmem_st32(o_col + cc * 32, raw);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc)
+            tmem_st32(o_col + cc * 32, *reinterpret_cast<const uint32_t(*)[32]>(raw + 32 * cc));
         }
         if (PNQ) {
           const uint32_t lv = tmem_ld1(l_col);
@@ -569,8 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
     if (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag,
-                                             p.status, kStatusTimeoutPV | 1));
+      ok = warp_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
+                     kStatusTimeoutPV | 1);
     }
     if (ok) {
       tc_fence_after();
@@ -621,16 +726,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool PNQ, bool DBG, bool NV>
+template <int D, int PM, bool DBG, bool NV>
 static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PNQ, DBG, NV>,
+  // the softmax warpgroups' register increase is served from the block's launch allocation: a
+  // build with fewer registers per thread than the split assumes would make it wait forever
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t ea = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, PM, DBG, NV>);
+    if (ea != cudaSuccess) return ea;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PM, DBG, NV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned n_units = static_cast<unsigned>((p.Npad / kBM + 1) / 2);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * n_units;
-  mxattn_fwd_kernel<D, PNQ, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
@@ -638,10 +753,15 @@ template <int D, bool NV>
 static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const bool dbg = p.dbg_codes != nullptr;
-  if (p.pnq) return dbg ? launch_k<D, true, true, NV>(tmQ, tmK, tmV, p, stream)
-                        : launch_k<D, true, false, NV>(tmQ, tmK, tmV, p, stream);
-  return dbg ? launch_k<D, false, true, NV>(tmQ, tmK, tmV, p, stream)
-             : launch_k<D, false, false, NV>(tmQ, tmK, tmV, p, stream);
+  if (p.pnq == 2) {
+    if constexpr (NV) return cudaErrorInvalidValue;    // the exp-free rule is MXFP4 only
+    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, p, stream)
+                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, p, stream);
+  }
+  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, p, stream)
+                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, p, stream);
+  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, p, stream)
+             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, p, stream);
 }
 
 template <int D>

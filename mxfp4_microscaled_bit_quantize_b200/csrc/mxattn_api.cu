@@ -213,7 +213,7 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   p.rows_per_head = src.rows_per_head;
   p.causal = causal ? 1 : 0;
   p.mode = scale_mode;
-  p.pnq = pnq ? 1 : 0;
+  p.pnq = pnq;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   p.status = status ? status : reinterpret_cast<unsigned int*>(w);
   p.dbg_codes = p_codes;
@@ -239,6 +239,14 @@ mxattn_status check_forward_args(const void* q, const void* k, const void* v, co
   if (out && !aligned(out, 16)) return MXATTN_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256)) return MXATTN_ERR_INVALID_ARG;
   if (ws_bytes < L->total) return MXATTN_ERR_WORKSPACE;
+  return MXATTN_OK;
+}
+
+// The rule of the P~ operand (the `pnq` argument): MXATTN_P_CONVENTIONAL, MXATTN_P_PNQ or
+// MXATTN_P_EFQ; the exp-free rule is defined for power-of-two (MXFP4) block scales only.
+mxattn_status check_p_rule(int pnq, int scale_mode) {
+  if (pnq < MXATTN_P_CONVENTIONAL || pnq > MXATTN_P_EFQ) return MXATTN_ERR_INVALID_ARG;
+  if (pnq == MXATTN_P_EFQ && scale_mode == MXATTN_SCALE_NVFP4) return MXATTN_ERR_UNSUPPORTED;
   return MXATTN_OK;
 }
 
@@ -450,6 +458,7 @@ mxattn_status mxattn_forward_attend(void* out, int B, int Hq, int Hkv, int N, in
   WsLayout L;
   mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, out, B, Hq, Hkv, N, d, scale_mode, out_dtype,
                                        workspace, workspace_bytes, &L);
+  if (s == MXATTN_OK) s = check_p_rule(pnq, scale_mode);
   if (s != MXATTN_OK) return s;
   return attend_impl(out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, workspace,
                      static_cast<cudaStream_t>(stream), L, workspace_codes(workspace, L), -1, 0, 0, nullptr,
@@ -465,6 +474,7 @@ mxattn_status mxattn_forward_quantized(const uint8_t* qc, const uint8_t* qs, con
   WsLayout L;
   mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, out, B, Hq, Hkv, N, d, p_scale_mode, out_dtype,
                                        workspace, workspace_bytes, &L);
+  if (s == MXATTN_OK) s = check_p_rule(pnq, p_scale_mode);
   if (s != MXATTN_OK) return s;
   if (p_scale_mode == MXATTN_SCALE_NVFP4) return MXATTN_ERR_UNSUPPORTED;   // MXFP4 operands only
   if (static_cast<uint64_t>(B) * Hq * N >= (1ull << 31)) return MXATTN_ERR_UNSUPPORTED;
@@ -499,6 +509,7 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
   WsLayout L;
   mxattn_status s = check_forward_args(q, k, v, out, B, Hq, Hkv, N, d, scale_mode, out_dtype, workspace,
                                        workspace_bytes, &L);
+  if (s == MXATTN_OK) s = check_p_rule(pnq, scale_mode);
   if (s != MXATTN_OK) return s;
   if (p_codes || p_scales) {
     if (!p_codes || !p_scales || dbg_bh < 0 || dbg_bh >= B * Hq || dbg_r0 < 0 || dbg_r1 <= dbg_r0 ||
@@ -601,6 +612,7 @@ mxattn_status mxattn_forward_host(const void* q, const void* k, const void* v, v
   mxattn_status s = check_forward_args(nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, N, d, scale_mode, out_dtype,
                                        workspace, workspace_bytes, &L);
   if (s != MXATTN_OK && s != MXATTN_ERR_WORKSPACE) return s;
+  if ((s = check_p_rule(pnq, scale_mode)) != MXATTN_OK) return s;
   HostPlan P;
   if (!host_plan(B, Hq, Hkv, N, d, out_dtype, &P)) return MXATTN_ERR_UNSUPPORTED;
   if (workspace_bytes < P.total) return MXATTN_ERR_WORKSPACE;

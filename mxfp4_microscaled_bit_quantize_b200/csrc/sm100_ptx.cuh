@@ -87,6 +87,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for a thread on a latency-critical path: it polls instead of suspending, so it reacts
+// within a few cycles of the phase completing. Same bounds and error reporting as mbar_wait (the
+// abort flag and the clock are read every 256 polls).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned int* status, unsigned int code) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        atomicCAS(status, 0u, code);
+        return false;
+      }
+    }
+  }
+}
+
 // True in exactly one lane of the (converged) warp; lets a warp-uniform loop issue
 // single-thread operations without a divergent branch around them.
 __device__ __forceinline__ bool elect_one_sync() {
@@ -289,6 +322,29 @@ __device__ __forceinline__ void ffma2_bc(float& r0, float& r1, float a0, float a
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
+// Packed general forms: (a0, a1) + (b0, b1) and (a0, a1) * (b0, b1) + (c0, c1).
+__device__ __forceinline__ void fadd2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 // Two fp32 products in one packed instruction: (a0, a1) * (b, b).
 __device__ __forceinline__ void fmul2_b(float& r0, float& r1, float a0, float a1, float b) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -298,6 +354,21 @@ __device__ __forceinline__ void fmul2_b(float& r0, float& r1, float a0, float a1
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(r0), "=f"(r1)
       : "f"(a0), "f"(a1), "f"(b));
+}
+
+// fma with the result clamped to [0, 1] (round to nearest, then saturate).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Nibble packing with saturation to [0, 15]: returns (acc << 8) | (hi << 4) | lo, hi and lo read
+// as signed 32-bit integers (negative values pack as 0).
+__device__ __forceinline__ uint32_t pack_u4x2(uint32_t acc, uint32_t hi, uint32_t lo) {
+  uint32_t d;
+  asm("cvt.pack.sat.u4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(hi), "r"(lo), "r"(acc));
+  return d;
 }
 
 // Named barrier ID (an immediate, so that the kernel reserves only the barriers it names) over
@@ -319,6 +390,17 @@ __device__ __forceinline__ bool bar_and(bool v) {
 template <int ID, int COUNT>
 __device__ __forceinline__ void bar_sync() {
   asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(COUNT) : "memory");
+}
+
+// Per-warpgroup register budget (all four warps of the warpgroup execute it). An increase waits
+// until other warpgroups have released enough of the registers the block was launched with.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // max(a, b, c) in one instruction (three-input form, sm_100+).

@@ -3,4 +3,4 @@
 TEST INFRASTRUCTURE ONLY: used by tests/, the package smoke check and the benchmark's
 CPU-baseline leg. The library never imports it and shares no code with it.
 """
-from . import mxfp4, attention  # noqa: F401
+from . import mxfp4, attention, efq  # noqa: F401

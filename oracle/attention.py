@@ -42,6 +42,9 @@ Readings taken where the pages are silent (each also listed in the design notes)
   its block amax, scale exponent and code are chosen. Everything else stays fp64.
 * Keys >= N and (causal) keys > i are masked: p = 0, code +0; an all-masked 32-key
   block gets scale byte 0x00.
+* pnq = 2 (P_EFQ) replaces exp-then-quantize by the exp-free rule of oracle/efq.py (EFQ-Softmax
+  abstract): the codes come from the base-2 shifted scores through one affine map, and that
+  operand feeds both the numerator and the denominator, as under PNQ. MXFP4 modes only.
 * mode = 2 (nvfp4.SCALE_NVFP4) is the NVFP4 comparison format of oracle/nvfp4.py for all four
   operands: blocks of 16 with E4M3 scales; P~ blocks are 16 keys, each decision again taken on
   the fp32-rounded P~ (scale byte from fp32(amax / 6), element from fp32(p / s)).
@@ -50,10 +53,13 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import efq
 from . import mxfp4 as mx
 from . import nvfp4 as nv
 
 KV_TILE = 128         # the library's documented tile width (MXATTN_KV_TILE)
+P_CONVENTIONAL, P_PNQ, P_EFQ = 0, 1, 2     # the `pnq` argument: rule of the P~ operand and row sum
+LOG2E = 1.0 / np.log(2.0)
 
 
 def dequantized_qkv(q, k, v, mode: int):
@@ -114,6 +120,9 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
     row_idx = np.asarray(row_idx, dtype=np.int64)
     N, d = kd.shape
     blk = block_size(mode)
+    rule = int(pnq)
+    if rule == P_EFQ and mode == nv.SCALE_NVFP4:
+        raise ValueError("the exp-free P~ rule is defined for MXFP4 (power-of-two block scales) only")
     assert kv_tile % mx.BLOCK == 0
     R = qd_rows.shape[0]
     sigma = 1.0 / np.sqrt(d)
@@ -127,6 +136,8 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
         rec_scales = np.zeros((R, npad // blk), dtype=np.uint8)
         rec_y = np.zeros((R, npad))
         rec_amax = np.zeros((R, npad // blk))
+        rec_z = np.full((R, npad), -np.inf)
+        rec_zmag = np.zeros((R, npad))
     for t in range(n_tiles):
         j0 = t * kv_tile
         keys = np.arange(j0, j0 + kv_tile)
@@ -144,10 +155,29 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
         with np.errstate(invalid="ignore"):
             alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))
             p = np.where(mask, 0.0, np.exp(s - m_new[:, None]))
-        if quantize_p:
+        if quantize_p and rule == P_EFQ:
+            with np.errstate(invalid="ignore"):
+                u = np.where(mask, -np.inf, (s - m_new[:, None]) * LOG2E)   # log2 P~
+            qv, codes, sbytes, z = efq.efq_quantize_p(u, mode)
+            denom = qv
+            if record_p:
+                rec_codes[:, j0:j0 + kv_tile] = codes
+                nb0 = j0 // blk
+                rec_scales[:, nb0:nb0 + kv_tile // blk] = sbytes
+                rec_z[:, j0:j0 + kv_tile] = z
+                # magnitude of the terms that form 2 r + 2 (scores, running max, block exponent):
+                # the scale of the fp32 rounding a kernel makes in it
+                e_el = np.repeat(sbytes.astype(np.float64) - mx.E8M0_BIAS, blk, axis=1)
+                with np.errstate(invalid="ignore"):
+                    rec_zmag[:, j0:j0 + kv_tile] = 2.0 * (np.abs(np.where(mask, 0.0, s)) + np.abs(m_new)[:, None]) \
+                        * LOG2E + 2.0 * np.abs(e_el) + 2.0
+                with np.errstate(over="ignore"):
+                    rec_amax[:, nb0:nb0 + kv_tile // blk] = np.exp2(u.reshape(R, -1, blk).max(axis=-1)).astype(
+                        np.float32)
+        elif quantize_p:
             p32 = p.astype(np.float32)                     # decision precision: fp32
             qv, codes, sbytes = _quantize_p(p32, mode)
-            denom = qv if pnq else p32.astype(np.float64)
+            denom = qv if rule != P_CONVENTIONAL else p32.astype(np.float64)
             if record_p:
                 rec_codes[:, j0:j0 + kv_tile] = codes
                 nb0 = j0 // blk
@@ -171,7 +201,8 @@ def attention_rows(qd_rows, row_idx, kd, vd, *, causal: bool, mode: int, pnq: bo
         m = m_new
     out = acc / l[:, None]
     if record_p:
-        return out, dict(codes=rec_codes, scales=rec_scales, y=rec_y, amax=rec_amax)
+        return out, dict(codes=rec_codes, scales=rec_scales, y=rec_y, amax=rec_amax, z=rec_z, zmag=rec_zmag,
+                         rule=rule)
     return out
 
 

@@ -5,7 +5,9 @@ Tolerances (fixed before measurement):
   * Q/K/V codes and scales: bit-exact (a pure function of the bf16 input).
   * P~ codes: mismatch rate <= 1e-4, and every mismatch must sit at a rounding tie the
     fp32 arithmetic can flip: the oracle's scaled value lies within TIE_REL of an E2M1
-    rounding midpoint, or the block amax lies within TIE_REL of a scale-exponent boundary.
+    rounding midpoint (for the exp-free rule: its argument 2 r + 2 lies within TIE_REL times
+    the magnitude of its terms of a half-integer), or the block amax lies within TIE_REL of a
+    scale-exponent boundary.
     TIE_REL = 2^-15 covers the GPU's independent error sources (fp32 score accumulation in
     the tensor core, the fp32 exponent argument, ex2.approx), each a few fp32 ulps of an
     argument of magnitude up to ~100.
@@ -51,6 +53,15 @@ def near_scale_boundary(amax: np.ndarray, mode: int) -> np.ndarray:
     return out
 
 
+def near_half_integer(z: np.ndarray, zmag: np.ndarray) -> np.ndarray:
+    """Exp-free rule: the argument 2 r + 2 lies within TIE_REL * (magnitude of its terms) of a
+    rounding boundary n + 1/2, where the kernel's fp32 arithmetic can take the other side."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(invalid="ignore"):
+        d = np.abs(z - np.floor(z) - 0.5)
+    return np.isfinite(z) & (d <= TIE_REL * np.asarray(zmag, dtype=np.float64))
+
+
 def classify_p_mismatches(gpu_codes, gpu_scales, rec, mode, n_valid):
     """Compare GPU P~ dumps with the oracle's record for the same rows.
 
@@ -67,7 +78,11 @@ def classify_p_mismatches(gpu_codes, gpu_scales, rec, mode, n_valid):
     blk = np.repeat(np.arange(nb_valid), bs)[:n_valid]
     scale_mis_blk = gs != os_
     explained_blk = near_scale_boundary(rec["amax"][:, :nb_valid], mode)
-    explained = near_midpoint(rec["y"][:, :n_valid]) | explained_blk[:, blk]
+    if rec.get("rule", 1) == 2:
+        near = near_half_integer(rec["z"][:, :n_valid], rec["zmag"][:, :n_valid])
+    else:
+        near = near_midpoint(rec["y"][:, :n_valid])
+    explained = near | explained_blk[:, blk]
     unexplained = (code_mis & ~explained) | (scale_mis_blk & ~explained_blk)[:, blk]
     return dict(rate=float(code_mis.mean()), n=int(code_mis.size), mismatches=int(code_mis.sum()),
                 unexplained=int(unexplained.sum()), scale_mismatch_blocks=int(scale_mis_blk.sum()))

@@ -141,6 +141,11 @@ def test_forward_argument_checks(lib):
     assert call(q=FAKE + 2) == INVALID
     assert call(ws=FAKE + 16) == INVALID
     assert call(wsb=good - 1) == WORKSPACE
+    # the P~ rule: conventional, PNQ or exp-free; the exp-free rule needs power-of-two scales
+    assert call(pnq=3) == INVALID
+    assert call(pnq=-1) == INVALID
+    assert call(pnq=2, mode=2) == UNSUPPORTED
+    assert call(pnq=2, wsb=good - 1) == WORKSPACE      # accepted up to the workspace check
 
 
 def test_forward_quantized_argument_checks(lib):

@@ -14,7 +14,8 @@ from oracle import mxfp4 as mx
 from tests import parity
 
 pytestmark = pytest.mark.gpu
-MODES = [(mx.SCALE_UOS, True), (mx.SCALE_OCP, False), (mx.SCALE_UOS, False), (mx.SCALE_OCP, True)]
+MODES = [(mx.SCALE_UOS, True), (mx.SCALE_OCP, False), (mx.SCALE_UOS, False), (mx.SCALE_OCP, True),
+         (mx.SCALE_UOS, oa.P_EFQ), (mx.SCALE_OCP, oa.P_EFQ)]
 
 
 @pytest.fixture(scope="module")
@@ -85,6 +86,14 @@ def test_tiny_workload_all_modes(dev, mode, pnq):
 def test_shapes(dev, N, d, causal):
     q, k, v = _rand_qkv(1, 4, 2, N, d, seed=N + d + causal, qk_scale=1.5)
     _run_and_check(dev, q, k, v, causal, mx.SCALE_UOS, True, [(0, 0), (0, 3)])
+
+
+@pytest.mark.parametrize("N", [1, 100, 129, 300, 511])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_shapes_exp_free(dev, N, d, causal):
+    q, k, v = _rand_qkv(1, 4, 2, N, d, seed=1000 + N + d + causal, qk_scale=1.5)
+    _run_and_check(dev, q, k, v, causal, mx.SCALE_UOS, oa.P_EFQ, [(0, 0), (0, 3)])
 
 
 def test_gqa_and_batches(dev):
