@@ -247,19 +247,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: (b, kv head g, query head within group, pair of q tiles); the pair index runs
-  //      fastest so that co-scheduled CTAs share one KV head in L2; causal runs the longest first.
+  // ---- work unit: (b, kv head g, query head within group, pair of q tiles). Non-causal: the pair
+  //      index runs fastest, so that co-scheduled CTAs share one KV head in L2. Causal: units are
+  //      ordered by length across all heads, longest first (the head index runs fastest, so that
+  //      the CTAs in flight still cover few KV groups); the block scheduler's in-order dispatch then
+  //      gives each SM the longest unit left, and the last wave holds the shortest ones.
   const int n_qt = p.Npad / kBM;
   const int n_units = (n_qt + 1) / 2;
   const int group = p.Hq / p.Hkv;
-  int idx = blockIdx.x;
-  int unit = idx % n_units;
-  idx /= n_units;
-  const int bh_q = idx;                       // b * Hq + h  (h = g * group + hh)
-  const int b = idx / p.Hq;
-  const int h = idx % p.Hq;
+  const int n_bh = p.B * p.Hq;
+  int unit, bh_q;
+  if (p.causal) {
+    unit = n_units - 1 - static_cast<int>(blockIdx.x / n_bh);
+    bh_q = static_cast<int>(blockIdx.x % n_bh);
+  } else {
+    unit = static_cast<int>(blockIdx.x % n_units);
+    bh_q = static_cast<int>(blockIdx.x / n_units);
+  }
+  const int b = bh_q / p.Hq;                  // bh_q = b * Hq + h  (h = g * group + hh)
+  const int h = bh_q % p.Hq;
   const int bh_kv = b * p.Hkv + h / group;
-  if (p.causal) unit = n_units - 1 - unit;
   const int n_kv_all = p.Npad / kBN;
   int qt_x[2], n_kv_x[2];
 #pragma unroll
