@@ -1,8 +1,8 @@
 """Benchmark: MXFP4 attention forward (UOS + PNQ) on the video-DiT-shaped workload.
 
 One step = one full pass of the hot path through the library's public C-ABI call
-mxattn_forward: quantize Q and K along d and V along keys (three quantizer launches), then the
-fused tcgen05 attention kernel, on B=1, H=40, N=32760, d=128, non-causal, seeded synthetic
+mxattn_forward: quantize Q and K along d and V along keys (one quantizer launch for all three),
+then the fused tcgen05 attention kernel, on B=1, H=40, N=32760, d=128, non-causal, seeded synthetic
 inputs resident in HBM. Inputs (3 x 335 MB of bf16) exceed the 126 MB L2, so no flush is needed.
 
 Multi-GPU (torchrun): every rank runs its own independent problem of the same shape (weak
@@ -518,7 +518,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     elems = B * Hq * N * d + 2 * B * Hkv * N * d
-    # algorithmic bytes of the three quantizer launches: bf16 in, packed codes + scales out
+    # algorithmic bytes of the quantization pass (Q, K, V): bf16 in, packed codes + scales out
     quant_bytes = elems * 2 + elems // 2 + elems // 32
     qa_elems = xq0_numel
     qa_bytes = qa_elems * 2 + qa_elems // 2 + qa_elems // 32
@@ -581,7 +581,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                 "copy_floor": {"ms": copy_ms, "gbs": (h2d + d2h) / (copy_ms * 1e-3) / 1e9,
                                "frac": copy_ms / e2e_ms,
                                "note": "the same H2D and D2H bytes copied concurrently, no kernels"}},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 2 * args.steps,      # per step: the fused Q/K/V quantizer and the attention kernel
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:

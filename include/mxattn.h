@@ -118,7 +118,7 @@ size_t mxattn_forward_workspace_size(int B, int Hq, int Hkv, int N, int d);
  *   Supported: d in {64, 128}, 1 <= N, B*Hq*ceil(N/128) < 2^31.
  *   workspace: device memory of at least mxattn_forward_workspace_size(...) bytes, 256-byte
  *   aligned; its contents on entry are ignored; it must not be used concurrently by another
- *   call. The call runs the quantizer three times (Q, K, V^T) and then the fused kernel.
+ *   call. The call runs one quantizer launch (Q, K and V^T) and then the fused kernel.
  */
 mxattn_status mxattn_forward(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
                              int N, int d, int causal, int scale_mode, int pnq, int out_dtype,

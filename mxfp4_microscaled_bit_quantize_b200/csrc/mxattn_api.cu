@@ -136,7 +136,7 @@ mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, i
     if (launch_quantize_cols_nvfp4(vq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
     return MXATTN_OK;
   }
-  RowQuantParams rq{};
+  RowQuantParams rq{}, rk{};
   rq.x = static_cast<const __nv_bfloat16*>(q);
   rq.heads = static_cast<uint32_t>(B * Hq);
   rq.rows = static_cast<uint32_t>(N);
@@ -148,13 +148,12 @@ mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, i
   rq.mode = scale_mode;
   rq.sf_layout = kSfAtom;
   rq.vec_ok = aligned(q, 16) ? 1 : 0;
-  if (launch_quantize_rows(rq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
-  rq.x = static_cast<const __nv_bfloat16*>(k);
-  rq.heads = static_cast<uint32_t>(B * Hkv);
-  rq.codes = w + L.kc;
-  rq.scales = w + L.ks;
-  rq.vec_ok = aligned(k, 16) ? 1 : 0;
-  if (launch_quantize_rows(rq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  rk = rq;
+  rk.x = static_cast<const __nv_bfloat16*>(k);
+  rk.heads = static_cast<uint32_t>(B * Hkv);
+  rk.codes = w + L.kc;
+  rk.scales = w + L.ks;
+  rk.vec_ok = aligned(k, 16) ? 1 : 0;
   ColQuantParams cq{};
   cq.x = static_cast<const __nv_bfloat16*>(v);
   cq.heads = static_cast<uint32_t>(B * Hkv);
@@ -166,7 +165,8 @@ mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, i
   cq.mode = scale_mode;
   cq.sf_layout = kSfAtom;
   cq.vec_ok = aligned(v, 16) ? 1 : 0;
-  if (launch_quantize_cols(cq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
+  // one launch for all three operands
+  if (launch_quantize_qkv(rq, rk, cq, st) != cudaSuccess) return MXATTN_ERR_CUDA;
   (void)ws_bytes;
   return MXATTN_OK;
 }

@@ -44,6 +44,15 @@ struct ColQuantParams {
 cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream);
 cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream);
 
+// Q and K (row quantizer) and V (transposing quantizer) of one attention call in a single launch.
+struct QkvQuantParams {
+  RowQuantParams q, k;
+  ColQuantParams v;
+  uint32_t v_ctas, v_gx, v_gy;    // the transposing quantizer's CTAs come first, grid (v_gx, v_gy, heads)
+};
+cudaError_t launch_quantize_qkv(const RowQuantParams& q, const RowQuantParams& k, const ColQuantParams& v,
+                               cudaStream_t stream);
+
 // NVFP4 (blocks of 16, E4M3 scales) along the contiguous axis: codes [heads*rows][ceil(cols/16)*8],
 // scales [heads*rows][ceil(cols/16)].
 // With sf_layout = kSfAtom: rows [rows, rows_pad) are zero (codes 0, scale 0) and the scales go to

@@ -7,14 +7,16 @@
 // nearest-even on the E2M1 grid, saturating at 6, by the hardware conversion
 // cvt.rn.satfinite.e2m1x2.f32.
 //
-// Two kernels:
+// Kernels:
 //  * quantize_rows_kernel: blocks along the contiguous axis (Q, K, the standalone tensor). One
 //    thread owns one whole block: four 16-byte loads, a thread-local amax, one 16-byte store of
 //    codes. A warp therefore reads 2 KiB and writes 512 B of codes per step, fully coalesced.
 //  * quantize_cols_kernel: blocks along the row axis of a [R, C] matrix, written transposed as
-//    [C, R/2] codes (V along keys). A CTA stages 256 rows x 64 columns in shared memory; each
-//    thread then quantizes two consecutive 32-row blocks of one column and writes 32 contiguous
-//    bytes of codes.
+//    [C, R/2] codes (V along keys). Each thread loads two adjacent columns of 64 rows straight
+//    from global memory (4-byte loads, 128 contiguous bytes per warp load), quantizes the four
+//    32-row blocks and writes 32 contiguous bytes of codes per column.
+//  * quantize_qkv_kernel: both of the above for one attention call (Q and K along d, V
+//    transposed) in a single launch, so that the whole quantization pass is one kernel.
 //
 // Scale placement: row-major [.., rows, blocks] (the library's canonical layout), or the tile
 // layout the block-scaled tensor-core MMA consumes: per 128-row tile and 4 blocks along K, a
@@ -38,6 +40,12 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float* v) {
     v[2 * i] = __uint_as_float(w[i] << 16);
     v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
 }
 
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
@@ -64,114 +72,139 @@ __device__ __forceinline__ uint32_t quantize_block32(float* v, int mode, uint4& 
   return byte;
 }
 
+// One 32-element block (global block index g over heads x rows_pad x kb) of the row quantizer.
+__device__ __forceinline__ void quantize_rows_block(const RowQuantParams& p, uint32_t g) {
+  const uint32_t row_bytes = p.kb * 16u;
+  const uint32_t row = g / p.kb;               // head * rows_pad + n
+  const uint32_t kbi = g - row * p.kb;
+  const uint32_t head = row / p.rows_pad;
+  const uint32_t n = row - head * p.rows_pad;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = 0.f;
+  if (n < p.rows) {
+    const uint64_t src_row = static_cast<uint64_t>(head) * p.rows + n;
+    const __nv_bfloat16* src = p.x + src_row * p.cols + static_cast<uint64_t>(kbi) * 32u;
+    const uint32_t c0 = kbi * 32u;
+    if (p.vec_ok && c0 + 32u <= p.cols) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bf16x8_to_f32(ld_stream_u4(src + 8 * c), v + 8 * c);
+    } else {
+      for (uint32_t i = 0; i < 32u && c0 + i < p.cols; ++i) v[i] = __bfloat162float(src[i]);
+    }
+  }
+  uint4 codes;
+  const uint32_t byte = quantize_block32(v, p.mode, codes);
+  *reinterpret_cast<uint4*>(p.codes + static_cast<uint64_t>(row) * row_bytes + kbi * 16u) = codes;
+  uint64_t so;
+  if (p.sf_layout == kSfRowMajor) {
+    so = static_cast<uint64_t>(row) * p.kb + kbi;
+  } else {
+    const uint32_t tiles = p.rows_pad >> 7;
+    const uint32_t katoms = (p.kb + 3u) >> 2;
+    const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (n >> 7)) * katoms + (kbi >> 2);
+    so = atom * 512u + atom_offset(n & 127u, kbi & 3u);
+  }
+  p.scales[so] = static_cast<uint8_t>(byte);
+}
+
 __global__ void __launch_bounds__(256) quantize_rows_kernel(RowQuantParams p) {
   const uint32_t total = p.heads * p.rows_pad * p.kb;   // blocks
-  const uint32_t row_bytes = p.kb * 16u;
-  for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x) {
-    const uint32_t row = g / p.kb;               // head * rows_pad + n
-    const uint32_t kbi = g - row * p.kb;
-    const uint32_t head = row / p.rows_pad;
-    const uint32_t n = row - head * p.rows_pad;
-    float v[32];
+  for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x)
+    quantize_rows_block(p, g);
+}
+
+// quantize_cols_kernel: each thread owns two adjacent columns (channels) and 64 rows (keys), i.e.
+// two 32-row blocks per column. It issues 64 independent 4-byte loads (one bf16 pair per row; a
+// warp's load covers 128 contiguous bytes of one row), then quantizes its four blocks and writes
+// 32 contiguous bytes of codes per column (whole 32-byte sectors) and the two scale bytes of each
+// column with one store. No shared memory and no CTA barrier: the loads of every warp are in
+// flight together. A CTA of 8 warps covers 256 rows x 128 columns (2 column groups x 4 row
+// groups); grid.y walks wider matrices in steps of 128 columns.
+constexpr int kColRowsPerThread = 64;
+constexpr int kColCtaRows = 256;
+constexpr int kColCtaCols = 128;
+
+// The work of one CTA (bx, by, bz) of the transposing quantizer.
+__device__ __forceinline__ void quantize_cols_cta(const ColQuantParams& p, uint32_t bx, uint32_t by, uint32_t bz) {
+  const uint32_t head = bz;
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t col = by * kColCtaCols + (warp & 1) * 64 + 2 * lane;   // this thread's first column
+  const uint32_t r0 = bx * kColCtaRows + (warp >> 1) * kColRowsPerThread;
+  const uint32_t blk0 = r0 >> 5;                      // absolute block index along rows
+  if (col >= p.cols || blk0 >= p.nblk) return;
+  const bool two = col + 1 < p.cols;
+  const __nv_bfloat16* src = p.x + static_cast<uint64_t>(head) * p.rows * p.cols + col;
+  // 4-byte loads need an even column count (then every (row, even column) pair is 4-byte aligned)
+  const bool vec = p.vec_ok && (p.cols % 2u == 0u);
+  uint32_t w[kColRowsPerThread];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = 0.f;
-    if (n < p.rows) {
-      const uint64_t src_row = static_cast<uint64_t>(head) * p.rows + n;
-      const __nv_bfloat16* src = p.x + src_row * p.cols + static_cast<uint64_t>(kbi) * 32u;
-      const uint32_t c0 = kbi * 32u;
-      if (p.vec_ok && c0 + 32u <= p.cols) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) bf16x8_to_f32(ld_stream_u4(src + 8 * c), v + 8 * c);
+  for (int i = 0; i < kColRowsPerThread; ++i) {
+    const uint32_t r = r0 + i;
+    w[i] = 0u;
+    if (r < p.rows) {
+      const __nv_bfloat16* e = src + static_cast<uint64_t>(r) * p.cols;
+      if (vec) {
+        w[i] = ld_stream_u32(e);
       } else {
-        for (uint32_t i = 0; i < 32u && c0 + i < p.cols; ++i) v[i] = __bfloat162float(src[i]);
+        w[i] = __bfloat16_as_ushort(e[0]);
+        if (two) w[i] |= static_cast<uint32_t>(__bfloat16_as_ushort(e[1])) << 16;
       }
     }
-    uint4 codes;
-    const uint32_t byte = quantize_block32(v, p.mode, codes);
-    *reinterpret_cast<uint4*>(p.codes + static_cast<uint64_t>(row) * row_bytes + kbi * 16u) = codes;
-    uint64_t so;
-    if (p.sf_layout == kSfRowMajor) {
-      so = static_cast<uint64_t>(row) * p.kb + kbi;
-    } else {
-      const uint32_t tiles = p.rows_pad >> 7;
-      const uint32_t katoms = (p.kb + 3u) >> 2;
-      const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (n >> 7)) * katoms + (kbi >> 2);
-      so = atom * 512u + atom_offset(n & 127u, kbi & 3u);
+  }
+  const bool second = blk0 + 1 < p.nblk;
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    if (cc == 1 && !two) break;
+    uint4 codes[2];
+    uint32_t bytes[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t x = w[32 * b + i];
+        v[i] = __uint_as_float(cc == 0 ? x << 16 : x & 0xFFFF0000u);
+      }
+      bytes[b] = quantize_block32(v, p.mode, codes[b]);
     }
-    p.scales[so] = static_cast<uint8_t>(byte);
+    const uint32_t c = col + cc;
+    uint8_t* dst = p.codes + (static_cast<uint64_t>(head) * p.cols + c) * (p.nblk * 16u) + blk0 * 16u;
+    reinterpret_cast<uint4*>(dst)[0] = codes[0];
+    if (second) reinterpret_cast<uint4*>(dst)[1] = codes[1];
+    if (p.sf_layout == kSfRowMajor) {
+      uint8_t* sc = p.scales + (static_cast<uint64_t>(head) * p.cols + c) * p.nblk + blk0;
+      sc[0] = static_cast<uint8_t>(bytes[0]);
+      if (second) sc[1] = static_cast<uint8_t>(bytes[1]);
+    } else {
+      // atom per (head, 128-row tile, 128-column group); MN index = column, K index = block; the
+      // two blocks are K indices blk0 & 3 and (blk0 & 3) + 1, adjacent bytes (blk0 is even)
+      const uint32_t tiles = p.nblk >> 2;             // nblk is a multiple of 4 here
+      const uint32_t cgroups = (p.cols + 127u) >> 7;
+      const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (blk0 >> 2)) * cgroups + (c >> 7);
+      uint8_t* sc = p.scales + atom * 512u + atom_offset(c & 127u, blk0 & 3u);
+      *reinterpret_cast<uint16_t*>(sc) = static_cast<uint16_t>(bytes[0] | ((second ? bytes[1] : 0u) << 8));
+    }
   }
 }
 
-// Stage: 256 rows x 64 columns of bf16, row pitch 72 elements (144 B) so that the column reads
-// of the compute phase (32 lanes on consecutive columns) hit distinct banks.
-constexpr int kColTileRows = 256;
-constexpr int kColTileCols = 64;
-constexpr int kColPitch = 72;
-
 __global__ void __launch_bounds__(256) quantize_cols_kernel(ColQuantParams p) {
-  __shared__ __align__(16) __nv_bfloat16 tile[kColTileRows * kColPitch];
-  const uint32_t head = blockIdx.z;
-  const uint32_t r0 = blockIdx.x * kColTileRows;      // first row (key) of this tile
-  const uint32_t c0 = blockIdx.y * kColTileCols;      // first column (channel)
-  const __nv_bfloat16* src = p.x + static_cast<uint64_t>(head) * p.rows * p.cols;
-  const int tid = threadIdx.x;
+  quantize_cols_cta(p, blockIdx.x, blockIdx.y, blockIdx.z);
+}
 
-  // Load: each pass covers 32 rows x 64 columns, one 16-byte vector per thread.
-#pragma unroll 4
-  for (int pass = 0; pass < kColTileRows / 32; ++pass) {
-    const uint32_t rr = pass * 32 + (tid >> 3);
-    const uint32_t cc = (tid & 7) * 8;
-    const uint32_t r = r0 + rr, c = c0 + cc;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (r < p.rows) {
-      const __nv_bfloat16* s = src + static_cast<uint64_t>(r) * p.cols + c;
-      if (p.vec_ok && c + 8 <= p.cols) {
-        raw = ld_stream_u4(s);
-      } else {
-        uint16_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (uint32_t i = 0; i < 8 && c + i < p.cols; ++i) h[i] = __bfloat16_as_ushort(s[i]);
-        raw.x = h[0] | (uint32_t(h[1]) << 16);
-        raw.y = h[2] | (uint32_t(h[3]) << 16);
-        raw.z = h[4] | (uint32_t(h[5]) << 16);
-        raw.w = h[6] | (uint32_t(h[7]) << 16);
-      }
-    }
-    *reinterpret_cast<uint4*>(&tile[rr * kColPitch + cc]) = raw;
+// Q and K along d and V transposed in one launch: CTAs [0, v_ctas) are the transposing
+// quantizer's grid (flattened), the rest walk the Q blocks and then the K blocks grid-stride.
+__global__ void __launch_bounds__(256) quantize_qkv_kernel(QkvQuantParams p) {
+  if (blockIdx.x < p.v_ctas) {
+    const uint32_t bx = blockIdx.x % p.v_gx, rest = blockIdx.x / p.v_gx;
+    quantize_cols_cta(p.v, bx, rest % p.v_gy, rest / p.v_gy);
+    return;
   }
-  __syncthreads();
-
-  // Compute: thread (column cl, pair kp) quantizes row blocks 2kp and 2kp+1 of its column.
-  const uint32_t cl = tid & 63;
-  const uint32_t kp = tid >> 6;
-  const uint32_t col = c0 + cl;
-  const uint32_t blk0 = (r0 >> 5) + 2 * kp;          // absolute block index along rows
-  if (col >= p.cols || blk0 >= p.nblk) return;
-  uint4 codes[2];
-  uint32_t bytes[2];
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    float v[32];
-    const uint32_t rb = (2 * kp + b) * 32;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[(rb + i) * kColPitch + cl]);
-    bytes[b] = quantize_block32(v, p.mode, codes[b]);
-  }
-  const bool second = blk0 + 1 < p.nblk;
-  uint8_t* dst = p.codes + (static_cast<uint64_t>(head) * p.cols + col) * (p.nblk * 16u) + blk0 * 16u;
-  reinterpret_cast<uint4*>(dst)[0] = codes[0];
-  if (second) reinterpret_cast<uint4*>(dst)[1] = codes[1];
-  if (p.sf_layout == kSfRowMajor) {
-    uint8_t* s = p.scales + (static_cast<uint64_t>(head) * p.cols + col) * p.nblk + blk0;
-    s[0] = static_cast<uint8_t>(bytes[0]);
-    if (second) s[1] = static_cast<uint8_t>(bytes[1]);
-  } else {
-    // atom per (head, 128-row tile, 128-column group); MN index = column, K index = block
-    const uint32_t tiles = p.nblk >> 2;               // nblk is a multiple of 4 here
-    const uint32_t cgroups = (p.cols + 127u) >> 7;
-    const uint64_t atom = (static_cast<uint64_t>(head) * tiles + (blk0 >> 2)) * cgroups + (col >> 7);
-    uint8_t* s = p.scales + atom * 512u + atom_offset(col & 127u, blk0 & 3u);
-    s[0] = static_cast<uint8_t>(bytes[0]);
-    if (second) s[1] = static_cast<uint8_t>(bytes[1]);
+  const uint32_t nq = p.q.heads * p.q.rows_pad * p.q.kb, nk = p.k.heads * p.k.rows_pad * p.k.kb;
+  const uint32_t stride = (gridDim.x - p.v_ctas) * blockDim.x;
+  for (uint32_t g = (blockIdx.x - p.v_ctas) * blockDim.x + threadIdx.x; g < nq + nk; g += stride) {
+    if (g < nq) quantize_rows_block(p.q, g);
+    else quantize_rows_block(p.k, g - nq);
   }
 }
 
@@ -331,10 +364,31 @@ cudaError_t launch_quantize_rows(const RowQuantParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_quantize_qkv(const RowQuantParams& q, const RowQuantParams& k, const ColQuantParams& v,
+                               cudaStream_t stream) {
+  QkvQuantParams p{q, k, v, 0, 0, 0};
+  p.v_gx = (v.nblk * 32u + kColCtaRows - 1) / kColCtaRows;
+  p.v_gy = (v.cols + kColCtaCols - 1) / kColCtaCols;
+  const uint64_t v_ctas = (v.heads == 0 || v.cols == 0 || v.nblk == 0)
+                              ? 0 : static_cast<uint64_t>(p.v_gx) * p.v_gy * v.heads;
+  const uint64_t row_blocks = static_cast<uint64_t>(q.heads) * q.rows_pad * q.kb +
+                              static_cast<uint64_t>(k.heads) * k.rows_pad * k.kb;
+  if (v_ctas + row_blocks == 0) return cudaSuccess;
+  if (v_ctas >= (1ull << 31) || row_blocks >= (1ull << 32)) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const uint64_t want = (row_blocks + 255) / 256;
+  const uint64_t cap = static_cast<uint64_t>(sms) * 8;
+  const uint64_t row_ctas = want < cap ? want : cap;
+  p.v_ctas = static_cast<uint32_t>(v_ctas);
+  quantize_qkv_kernel<<<static_cast<unsigned>(v_ctas + row_ctas), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_cols(const ColQuantParams& p, cudaStream_t stream) {
   if (p.heads == 0 || p.cols == 0 || p.nblk == 0) return cudaSuccess;
-  dim3 grid((p.nblk * 32u + kColTileRows - 1) / kColTileRows, (p.cols + kColTileCols - 1) / kColTileCols,
-            p.heads);
+  dim3 grid((p.nblk * 32u + kColCtaRows - 1) / kColCtaRows, (p.cols + kColCtaCols - 1) / kColCtaCols, p.heads);
   quantize_cols_kernel<<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
