@@ -21,15 +21,17 @@
 // S(A, t+1), ... . Their softmax warps therefore run half a step apart, and on every SM
 // sub-partition one tile's serial work (S load, maxima, scale selection, stores, rescale) overlaps
 // the other tile's exponentials on the MUFU.
-// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 72 registers
-// per thread and each softmax warpgroup 216):
-//   warp 0     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
+// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 104 registers
+// per thread and each softmax warpgroup 200):
+//   warp 2     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
 //              an NSTAGE-deep shared-memory ring (mbarrier complete_tx).
-//   warps 2, 3 no role (they complete the control warpgroup).
-//   warp 1     TMEM owner and MMA issuer (one thread): copies scale atoms to TMEM with tcgen05.cp
-//              and issues, per key tile t, S(A, t+1), O_A += P~_A(t) V(t) (+ L_A), S(B, t+1),
-//              O_B += P~_B(t) V(t) (+ L_B). Each S waits until the previous user of the S buffer
-//              holds its scores in registers.
+//   warp 1     TMEM owner and S issuer (one thread): copies the Q and K scale atoms and issues
+//              S(A, t), S(B, t), S(A, t+1), ..., each once the previous user of the S buffer holds
+//              its scores in registers.
+//   warps 0, 3 P~V issuers of tiles A and B (one thread each): copy the P~ and V scale atoms to
+//              TMEM and issue O_X += P~_X(t) V(t) and L_X += P~_X(t) 1 as soon as tile X's softmax
+//              hands P~ over. The four control warps sit on the four SM sub-partitions, so that the
+//              tcgen05 issue work is spread next to all eight softmax warps, which set the pace.
 //   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per query row (TMEM lane = row).
 //              Per key tile a thread reads its 128 scores with tcgen05.ld, releases S, updates the
 //              running max, computes P~ / 2^e per 32-key block, quantizes it in registers, writes
@@ -62,7 +64,7 @@ constexpr int kThreads = 384;     // warpgroup 0: producer, MMA, 2 idle; warpgro
 // Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for 384
 // threads); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to kSoftmaxRegs.
 // The three shares add up to exactly the launch total, which the host checks before launching.
-constexpr int kLaunchRegs = 168, kCtlRegs = 72, kSoftmaxRegs = 216;
+constexpr int kLaunchRegs = 168, kCtlRegs = 104, kSoftmaxRegs = 200;
 static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 X, L_X at kColL + 16 X
@@ -70,11 +72,11 @@ constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 
 //   Q_X         kColSfQ + 8 X
 //   K of tile t kColSfK + 8 (t & 1)      V of tile t kColSfV + 8 (t & 1)
 //   P~_X(t)     kColSfP + 16 X + 8 (t & 1)
-//   ones        kColSf1
+//   ones        kColSf1 + 4 X (one copy per P~V issuer)
 // tcgen05.cp into columns an earlier MMA still reads is not ordered behind that MMA; the K, V and
 // P~ sets alternate by tile parity, and the set written for tile t was last read by a product of
 // tile t - 2, which the issuing thread has seen complete by then (see the MMA issuer).
-constexpr uint32_t kColSfQ = 416, kColSfK = 432, kColSfV = 448, kColSfP = 464, kColSf1 = 496;
+constexpr uint32_t kColSfQ = 416, kColSfK = 432, kColSfV = 448, kColSfP = 464, kColSf1 = 496;   // + 4 x
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
 constexpr int kPRowBytes = kBN / 2;                  // 64 bytes of codes per P~ / V^T row
 
@@ -113,7 +115,8 @@ struct __align__(1024) Smem {
   // for tile t.
   uint64_t bar_p_full[2][2];
   uint64_t bar_pv_done[2][2];             // completions of PV of query tile X, even / odd key tiles
-  uint64_t bar_drain;
+  uint64_t bar_drain[3];                  // each issuing warp's own final drain
+  uint64_t bar_ones;                      // the ones operand is in shared memory (PNQ)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -161,14 +164,10 @@ __device__ __forceinline__ void exp2_codes_poly(float& y0, float& y1, float x0, 
   y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
-// Wait of a whole warp for an mbarrier phase (bounded, see mbar_wait). kSpin polls instead of
-// suspending: the MMA issuer uses it under the exp-free rule, where the softmax phase is short and
-// the S-buffer hand-over (softmax release -> MMA issue -> next softmax) sets the pace.
-template <bool kSpin = false>
+// Wait of a whole warp for an mbarrier phase (bounded, see mbar_wait).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* status, unsigned int code) {
-  if constexpr (kSpin) return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, status, code));
-  else return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, code));
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, code));
 }
 
 // E8M0 byte of a P~ block maximum amax in [0, 1] (the running max bounds every P~ by 1): the OCP
@@ -181,11 +180,15 @@ __device__ __forceinline__ uint32_t p_scale_byte(float amax, int mode) {
   return static_cast<uint32_t>(max(byte, 0));
 }
 
-// Every kPolyEvery-th pair of keys takes its PNQ exponentials from exp2_codes_poly instead of the
-// MUFU (0: all on the MUFU). Measured on the video-DiT workload with 1/8, 1/4 and 1/2 of the
-// exponentials moved: no gain, because the MUFU is not what bounds the kernel (the exp-free rule,
-// which needs no exponential at all, runs only about a fifth faster); kept off.
-constexpr int kPolyEvery = 0;
+// kPolyPairs of the 16 key pairs of every 32-key chunk take their PNQ exponentials from
+// exp2_codes_poly (FMA and integer pipes) instead of the MUFU, spread evenly over the chunk. With
+// the tcgen05 issue work spread over all four SM sub-partitions the softmax warps set the pace and
+// the MUFU (16 results per clock per SM) is their busiest unit; measured on the video-DiT workload,
+// 4, 5, 6 and 7 of 16 pairs gave +2%, +7%, +3% and +1% over none.
+constexpr int kPolyPairs = 5;
+__host__ __device__ constexpr bool poly_pair(int pair) {
+  return ((pair + 1) * kPolyPairs) / 16 > (pair * kPolyPairs) / 16;
+}
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight copies / MMAs).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.bar_q, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&s.bar_kv_full[i], 1);
-      mbar_init(&s.bar_kv_empty[i], 1);
+      mbar_init(&s.bar_kv_empty[i], 2);    // one release per P~V issuer
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s.bar_s_full[x], 1);
@@ -291,7 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     mbar_init(&s.bar_s_empty, 4);
-    mbar_init(&s.bar_drain, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&s.bar_drain[i], 1);
+    mbar_init(&s.bar_ones, 1);
     s.abort_flag = 0;
     fence_mbar_init();
   }
@@ -307,7 +311,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
    regs_dec<kCtlRegs>();
-   if (warp == 0) {
+   // Two issuing warps on different SM sub-partitions share the tcgen05 work: warp 1 the S
+   // products (the latency-critical hand-overs of the S buffer), warp 0 the TMA loads and the
+   // P~V and row-sum products. Each waits on the barriers that gate its own products; the
+   // scale-atom sets stay safe as argued beside each copy below.
+   const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
+   auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
+   // Shared-memory descriptors: only the 14-bit start-address field (16-byte units) differs between
+   // the operands of one kind, so each is one OR of a fixed upper part with an address.
+   const uint64_t d_qk = smem_desc(0, 0, C::kQKSbo, C::kQKLayout);          // Q and K tiles
+   const uint64_t d_pv = smem_desc(0, 0, 8 * kPRowBytes, kLayoutSw64);      // P~, V^T and ones tiles
+   const uint32_t a_q = smem_u32(s.q[0]) >> 4, a_k = smem_u32(s.k[0]) >> 4, a_v = smem_u32(s.v[0]) >> 4;
+   const uint32_t a_p = smem_u32(s.p[0][0]) >> 4, a_ones = smem_u32(s.ones) >> 4;
+   if (warp == 2) {
     // ============================ TMA producer ============================
     // The whole warp runs the loop (warp-uniform operands); one elected lane issues the copies.
     const bool leader = elect_one_sync();
@@ -326,10 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     for (int t = 0; t < n_kv_max; ++t) {
       const int st = t % NS;
-      if (t >= NS) {
-        if (!warp_wait(&s.bar_kv_empty[st], ((t / NS) & 1) ^ 1, abort_flag, p.status, kStatusTimeoutEmpty | st))
-          break;
-      }
+      if (t >= NS &&
+          !warp_wait(&s.bar_kv_empty[st], ((t / NS) & 1) ^ 1, abort_flag, p.status, kStatusTimeoutEmpty | st))
+        break;
       if (leader) {
         mbar_arrive_expect_tx(&s.bar_kv_full[st], C::kKTileBytes + C::kVTileBytes + kQKSfBytes + kPVSfBytes);
         tma_load_2d(s.k[st], &tmK, &s.bar_kv_full[st], 0, bh_kv * p.rows_per_head + t * kBN);
@@ -351,29 +366,102 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(&s.bar_kv_full[t % NS], (t / NS) & 1);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ============================ MMA issuer ============================
-    // The whole warp runs the loop (warp-uniform descriptors); one elected lane issues every
-    // tcgen05 operation and commit, so completion tracking stays with that thread.
-    //
-    // Order per key tile t: S(A, t+1), PV(A, t), S(B, t+1), PV(B, t). A commit arrives only when
-    // every earlier operation of this thread has completed, so once this thread has seen the
-    // consumer of some S(X, t') (or PV) commit, every operation issued before that one is
-    // complete too. That gives the scale-atom sets their safety: the K set of tile t is written
-    // after the S buffer's previous user read its scores (so the S products of tile t - 2, issued
-    // earlier, are done); the V and P~ sets of tile t are written after PV(X, t)'s softmax has read
-    // S(X, t), which was issued after every product of tile t - 2.
-    const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
-    auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
+   } else if (warp == 0 || warp == 3) {
+    // ======================= P~V issuer of query tile x (warp 0: A, warp 3: B) =======================
+    // One elected thread copies the P~ (and, for the first product of a key tile, the V) scale atoms
+    // to TMEM and issues O_x += P~_x(t) V(t) and L_x += P~_x(t) 1 once tile x's softmax hands P~
+    // over. A commit arrives only when every earlier operation of its thread has completed.
+    const int x = warp == 0 ? 0 : 1;
+    const bool leader = elect_one_sync();
+    const uint32_t ones_sf = tmem + kColSf1 + 4 * x;      // each issuer holds its own ones atom
     if (PNQ) {
-      // ones operand (row 0 = code 1.0 for every key, rows 1..15 = 0) with unit scales
-      uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
-      for (int i = lane; i < kOnesRows * kPRowBytes / 4; i += 32) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
-      uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
-      for (int i = lane; i < 512 / 4; i += 32) sw[i] = NV ? 0x38383838u : 0x7F7F7F7Fu;   // E4M3 / E8M0 1.0
-      fence_proxy_async_smem();
+      if (x == 0) {
+        // ones operand (row 0 = code 1.0 for every key, rows 1..15 = 0) with unit scales
+        uint32_t* ow = reinterpret_cast<uint32_t*>(s.ones);
+        for (int i = lane; i < kOnesRows * kPRowBytes / 4; i += 32) ow[i] = (i < kPRowBytes / 4) ? 0x22222222u : 0u;
+        uint32_t* sw = reinterpret_cast<uint32_t*>(s.onesf);
+        for (int i = lane; i < 512 / 4; i += 32) sw[i] = NV ? 0x38383838u : 0x7F7F7F7Fu;   // E4M3 / E8M0 1.0
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bar_ones);
+      }
+      bool ok1 = warp_wait(&s.bar_ones, 0, abort_flag, p.status, kStatusTimeoutQ | 1);
+      tc_fence_after();
+      if (ok1 && leader) tc_cp_sf(ones_sf, sf_desc(s.onesf));
+      __syncwarp();
+    }
+    const int n_own = x == 0 ? n_kv_x[0] : n_kv_x[1];
+    const int n_other = x == 0 ? n_kv_x[1] : n_kv_x[0];
+    bool ok = true;
+    for (int t = 0; ok && t < n_kv_max; ++t) {
+      const int st = t % NS;
+      const int pb = t & 1;
+      if (t >= n_own) {
+        // no product of this query tile reads key tile t: count this issuer's release of the stage
+        if (leader) mbar_arrive(&s.bar_kv_empty[st]);
+        __syncwarp();
+        continue;
+      }
+      ok = warp_wait(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status, kStatusTimeoutP);
+      if (!ok) break;
+      // The V scale atoms of key tile t are copied by its first product: PV(A, t), or PV(B, t) when
+      // tile A has no product there. The other issuer's PV(t) waits for that product (its commit
+      // covers the copy). Before the copy, the set's last readers PV(., t - 2) must be complete:
+      // this issuer's own was seen complete by its softmax (which reused the P~ buffer after it),
+      // the other issuer's is waited for here.
+      const bool first = (x == 0) || t >= n_other;
+      if (!first) {
+        ok = warp_wait(&s.bar_pv_done[0][pb], (t >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 2);
+      } else if (t >= 2 && t - 2 < n_other) {
+        ok = warp_wait(&s.bar_pv_done[x ^ 1][pb], ((t >> 1) - 1) & 1, abort_flag, p.status,
+                            kStatusTimeoutPV | 3);
+      }
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t sfp = tmem + kColSfP + 16 * x + 8 * pb;
+        const uint32_t sfv = tmem + kColSfV + 8 * pb;
+#pragma unroll
+        for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfp + 4 * a, sf_desc(s.psf[x][pb] + a * 512));
+        if (first) {
+#pragma unroll
+          for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfv + 4 * a, sf_desc(s.vsf[st] + a * 512));
+        }
+        const uint32_t o_col = tmem + kColO + 128 * x, l_col = tmem + kColL + 16 * x;
+        const uint32_t pa = a_p + (2 * x + pb) * ((kBM * kPRowBytes) >> 4), va = a_v + st * (C::kVTileBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 64; ++kk) {
+          const uint64_t ad = d_pv | (pa + kk * 2), bd = d_pv | (va + kk * 2), od = d_pv | (a_ones + kk * 2);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          if constexpr (NV) {
+            tc_mma_nvf4(o_col, ad, bd, idesc_nvf4(D), sfp + 4 * kk, sfv + 4 * kk, acc);
+            if (PNQ) tc_mma_nvf4(l_col, ad, od, idesc_nvf4(kOnesRows), sfp + 4 * kk, ones_sf, acc);
+          } else {
+            // keys 64 kk .. 64 kk + 63 are blocks 2 kk, 2 kk + 1 of the P~ and V^T scale atoms
+            tc_mma_mxf4(o_col, ad, bd, idesc_mxf4(D, 2 * kk, 2 * kk), sfp, sfv, acc);
+            if (PNQ) tc_mma_mxf4(l_col, ad, od, idesc_mxf4(kOnesRows, 2 * kk, 0), sfp, ones_sf, acc);
+          }
+        }
+        tc_commit(&s.bar_pv_done[x][pb]);
+        // this issuer's release of the stage: the S products that read its K tile were complete
+        // before this product's softmax could read S(x, t)
+        tc_commit(&s.bar_kv_empty[st]);
+      }
+      __syncwarp();
+    }
+    // every product / copy issued above must complete before TMEM is released
+    if (leader) {
+      tc_commit(&s.bar_drain[x]);
+      drain_wait(&s.bar_drain[x], 0);
     }
     __syncwarp();
+   } else if (warp == 1) {
+    // ======================= TMEM owner and S issuer =======================
+    // Order: S(A, t), S(B, t), S(A, t+1), ...: each waits until the previous user of the S buffer
+    // holds its scores in registers. A commit arrives only when every earlier operation of this
+    // thread has completed, so when this thread has seen the user of S(., t - 1) read it, the S
+    // products of tile t - 2 are complete: the K set of tile t, which they read, may be rewritten
+    // (before that wait: the wait that S(., t - 1) itself passed already implies it).
     const bool leader = elect_one_sync();
     bool ok = warp_wait(&s.bar_q, 0, abort_flag, p.status, kStatusTimeoutQ);
     if (ok) {
@@ -383,28 +471,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int a = 0; a < kQKAtoms; ++a) tc_cp_sf(tmem + kColSfQ + 8 * x + 4 * a, sf_desc(s.qsf[x] + a * 512));
         }
-        if (PNQ) tc_cp_sf(tmem + kColSf1, sf_desc(s.onesf));
       }
       __syncwarp();
     }
-    // Shared-memory descriptors: only the 14-bit start-address field (16-byte units) differs between
-    // the operands of one kind, so each is one OR of a fixed upper part with an address.
-    const uint64_t d_qk = smem_desc(0, 0, C::kQKSbo, C::kQKLayout);          // Q and K tiles
-    const uint64_t d_pv = smem_desc(0, 0, 8 * kPRowBytes, kLayoutSw64);      // P~, V^T and ones tiles
-    const uint32_t a_q = smem_u32(s.q[0]) >> 4, a_k = smem_u32(s.k[0]) >> 4, a_v = smem_u32(s.v[0]) >> 4;
-    const uint32_t a_p = smem_u32(s.p[0][0]) >> 4, a_ones = smem_u32(s.ones) >> 4;
     int s_uses = 0;      // S products issued so far (A and B alternate on the one buffer)
     auto issue_s = [&](int x, int t) -> bool {
       const int st = t % NS;
       const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
       const uint32_t sfk = tmem + kColSfK + 8 * (t & 1);
       if (first) {
-        if (!warp_wait<EFQ>(&s.bar_kv_full[st], (t / NS) & 1, abort_flag, p.status,
-                                            kStatusTimeoutKV | st))
+        if (!warp_wait(&s.bar_kv_full[st], (t / NS) & 1, abort_flag, p.status, kStatusTimeoutKV | st))
           return false;
-        // the K atoms of tile t go to the set the S products of tile t - 2 read; those completed
-        // before the S buffer's user of S(t - 1) could read it, which this thread waited for when it
-        // issued the S product that followed (or there was none)
         tc_fence_after();
         if (leader) {
 #pragma unroll
@@ -413,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the previous user of the S buffer must hold its scores in registers
       if (s_uses > 0 &&
-          !warp_wait<EFQ>(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
+          !warp_wait(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
         return false;
       tc_fence_after();
       if (leader) {
@@ -432,56 +509,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++s_uses;
       return true;
     };
-    auto issue_pv = [&](int x, int t) -> bool {
-      const int st = t % NS;
-      const int pb = t & 1;
-      if (!warp_wait<EFQ>(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status, kStatusTimeoutP))
-        return false;
-      tc_fence_after();
-      const bool first = (x == 0) || t >= n_kv_x[0];      // first product of key tile t
-      const bool last = (x == 1) || t >= n_kv_x[1];       // last reader of the tile's stage
-      if (leader) {
-        const uint32_t sfp = tmem + kColSfP + 16 * x + 8 * pb;
-        const uint32_t sfv = tmem + kColSfV + 8 * pb;
-#pragma unroll
-        for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfp + 4 * a, sf_desc(s.psf[x][pb] + a * 512));
-        if (first) {
-#pragma unroll
-          for (int a = 0; a < kPVAtoms; ++a) tc_cp_sf(sfv + 4 * a, sf_desc(s.vsf[st] + a * 512));
-        }
-        const uint32_t o_col = tmem + kColO + 128 * x, l_col = tmem + kColL + 16 * x;
-        const uint32_t pa = a_p + (2 * x + pb) * ((kBM * kPRowBytes) >> 4), va = a_v + st * (C::kVTileBytes >> 4);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 64; ++kk) {
-          const uint64_t ad = d_pv | (pa + kk * 2), bd = d_pv | (va + kk * 2), od = d_pv | (a_ones + kk * 2);
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (NV) {
-            tc_mma_nvf4(o_col, ad, bd, idesc_nvf4(D), sfp + 4 * kk, sfv + 4 * kk, acc);
-            if (PNQ) tc_mma_nvf4(l_col, ad, od, idesc_nvf4(kOnesRows), sfp + 4 * kk, tmem + kColSf1, acc);
-          } else {
-            // keys 64 kk .. 64 kk + 63 are blocks 2 kk, 2 kk + 1 of the P~ and V^T scale atoms
-            tc_mma_mxf4(o_col, ad, bd, idesc_mxf4(D, 2 * kk, 2 * kk), sfp, sfv, acc);
-            if (PNQ) tc_mma_mxf4(l_col, ad, od, idesc_mxf4(kOnesRows, 2 * kk, 0), sfp, tmem + kColSf1, acc);
-          }
-        }
-        tc_commit(&s.bar_pv_done[x][pb]);
-        if (last) tc_commit(&s.bar_kv_empty[st]);
-      }
-      __syncwarp();
-      return true;
-    };
     if (ok && n_kv_x[0] > 0) ok = issue_s(0, 0);
     if (ok && n_kv_x[1] > 0) ok = issue_s(1, 0);
-    for (int t = 0; ok && t < n_kv_max; ++t) {
+    for (int t = 0; ok && t + 1 < n_kv_max; ++t) {
       if (ok && t + 1 < n_kv_x[0]) ok = issue_s(0, t + 1);
-      if (ok && t < n_kv_x[0]) ok = issue_pv(0, t);
       if (ok && t + 1 < n_kv_x[1]) ok = issue_s(1, t + 1);
-      if (ok && t < n_kv_x[1]) ok = issue_pv(1, t);
     }
-    // every MMA / copy issued above must complete before TMEM is released
+    // every product / copy issued above must complete before TMEM is released
     if (leader) {
-      tc_commit(&s.bar_drain);
-      drain_wait(&s.bar_drain, 0);
+      tc_commit(&s.bar_drain[2]);
+      drain_wait(&s.bar_drain[2], 0);
     }
     __syncwarp();
    }
@@ -608,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; i += 2) {
             float x0, x1;
             ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
-            if (PM == 1 && !NV && kPolyEvery > 0 && (i / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+            if (PM == 1 && poly_pair(i / 2)) {
               exp2_codes_poly(y[i], y[i + 1], x0, x1);
             } else {
               y[i] = ex2_approx_ftz(x0);

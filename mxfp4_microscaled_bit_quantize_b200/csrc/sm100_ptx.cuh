@@ -100,26 +100,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// mbar_wait for a thread on a latency-critical path: it polls instead of suspending, so it reacts
-// within a few cycles of the phase completing. Same bounds and error reporting as mbar_wait (the
-// abort flag and the clock are read every 256 polls).
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                               unsigned int* status, unsigned int code) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        atomicCAS(status, 0u, code);
-        return false;
-      }
-    }
-  }
-}
-
 // True in exactly one lane of the (converged) warp; lets a warp-uniform loop issue
 // single-thread operations without a divergent branch around them.
 __device__ __forceinline__ bool elect_one_sync() {
