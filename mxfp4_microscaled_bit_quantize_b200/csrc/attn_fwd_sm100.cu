@@ -492,6 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (s_uses > 0 &&
           !warp_wait(&s.bar_s_empty, (s_uses - 1) & 1, abort_flag, p.status, kStatusTimeoutS))
         return false;
+      // tile x's softmax writes P~(x, t) into the buffer that P~V(x, t - 2) read: that product must be
+      // complete before S(x, t) is handed over (it is, long since, in the steady state; waiting here
+      // keeps the wait off the softmax warps' path)
+      if (t >= 2 && !warp_wait(&s.bar_pv_done[x][t & 1], ((t >> 1) - 1) & 1, abort_flag, p.status, kStatusTimeoutPV))
+        return false;
       tc_fence_after();
       if (leader) {
         const uint32_t qa = a_q + x * (C::kQTileBytes >> 4), ka = a_k + st * (C::kKTileBytes >> 4);
@@ -607,12 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (bb % 4 == 0) sbytes[bb / 4] = 0;
         sbytes[bb / 4] |= byte << (8 * (bb % 4));
       }
-      // P~ buffer t&1 is free once the product of key tile t-2 (its last reader) has completed
+      // P~ buffer t&1: its last reader, the product of key tile t-2, completed before S(x, t) was
+      // issued (the S issuer waits for it)
       const int pb = t & 1;
-      if (t >= 2) {
-        ok = warp_wait(&s.bar_pv_done[x][pb], ((t >> 1) - 1) & 1, abort_flag, p.status, kStatusTimeoutPV);
-        if (!ok) break;
-      }
       // 32 keys at a time: 16 packed FMAs, 32 ex2, four words of codes, one 16-byte store
       uint8_t* p_row = s.p[x][pb] + r * kPRowBytes;
       uint8_t* d_row = (DBG && dbg) ? p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) + t * kPRowBytes
