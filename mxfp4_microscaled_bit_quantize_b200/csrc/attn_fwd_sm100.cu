@@ -234,8 +234,11 @@ __device__ __forceinline__ float lg2_approx(float x) {
 template <int D, int PM, bool DBG, bool NV>
 __global__ void __launch_bounds__(kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                      const AttnParams p) {
   static_assert(PM >= 0 && PM <= 2 && !(NV && PM == 2), "P~ rule");
+  static_assert(offsetof(Smem<D>, p) % 1024 == 0 && sizeof(Smem<D>::p[0]) == 4 * 4096,
+                "the output stage needs four 1024-aligned 4 KB quarters per query tile");
   constexpr bool PNQ = PM != 0;     // the row sum is the ones-operand product of the quantized P~
   constexpr bool EFQ = PM == 2;
   using C = Cfg<D>;
@@ -730,37 +733,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_wait_ld();
       }
       const float inv_l = 1.f / l;
-      const bool store = qrow < p.N;
-      const size_t orow = (static_cast<size_t>(bh_q) * p.N + (store ? qrow : 0)) * D;
+      // The normalised rows leave through shared memory and tiled TMA stores, so that the global
+      // writes are whole lines: each warp stages a 32-row x 128-byte chunk (32 fp32 or 64 bf16
+      // columns) in its quarter of its query tile's P~ buffers, which no product reads any more
+      // once the last P~V product has completed. 128-byte swizzle: the 16-byte piece j of row r
+      // sits at position j ^ (r & 7), so the eight stores of a warp cover all banks. The tensor
+      // map is [B*Hq][N][D]: rows past N are clipped by the copy.
+      uint8_t* stage = s.p[x][0] + quarter * 4096;
+      const uint32_t row_addr = smem_u32(stage) + static_cast<uint32_t>(lane) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
+      const int y0 = qt * kBM + quarter * 32;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t raw[32];
         tmem_ld32(o_col + cc * 32, raw);
         tc_wait_ld();
-        if (store) {
-          if (p.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow + cc * 32);
+        const bool half2 = p.out_bf16 && (cc & 1);        // bf16: second half of a 128-byte row
+        if (cc > 0 && !half2) {                           // the previous chunk's copy has read the stage
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+        }
+        if (p.out_bf16) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t wv[4];
+          for (int v = 0; v < 4; ++v) {
+            uint32_t wv[4];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * u]) * inv_l,
-                                                                __uint_as_float(raw[v * 8 + 2 * u + 1]) * inv_l);
-                wv[u] = *reinterpret_cast<const uint32_t*>(&h2);
-              }
-              dst[v] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            for (int u = 0; u < 4; ++u) {
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * u]) * inv_l,
+                                                              __uint_as_float(raw[v * 8 + 2 * u + 1]) * inv_l);
+              wv[u] = *reinterpret_cast<const uint32_t*>(&h2);
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + cc * 32);
+            st_shared_v4(row_addr + ((((half2 ? 4u : 0u) + v) ^ sw) << 4), wv[0], wv[1], wv[2], wv[3]);
+          }
+        } else {
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(raw[4 * v]) * inv_l, __uint_as_float(raw[4 * v + 1]) * inv_l,
-                                   __uint_as_float(raw[4 * v + 2]) * inv_l,
-                                   __uint_as_float(raw[4 * v + 3]) * inv_l);
+          for (int v = 0; v < 8; ++v)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(v) ^ sw) << 4),
+                         __float_as_uint(__uint_as_float(raw[4 * v]) * inv_l),
+                         __float_as_uint(__uint_as_float(raw[4 * v + 1]) * inv_l),
+                         __float_as_uint(__uint_as_float(raw[4 * v + 2]) * inv_l),
+                         __float_as_uint(__uint_as_float(raw[4 * v + 3]) * inv_l));
+        }
+        if (!p.out_bf16 || half2) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (y0 < p.N) tma_store_3d(&tmO, stage, p.out_bf16 ? (cc >> 1) * 64 : cc * 32, y0, bh_q);
+            bulk_commit_group();
           }
         }
       }
+      // the stage must stay valid until the copies have read it
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
     }
     tc_fence_before();
   }
@@ -773,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int PM, bool DBG, bool NV>
-static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
   // the softmax warpgroups' register increase is served from the block's launch allocation: a
@@ -791,36 +816,37 @@ static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
   if (e != cudaSuccess) return e;
   const unsigned n_units = static_cast<unsigned>((p.Npad / kBM + 1) / 2);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * n_units;
-  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError();
 }
 
 template <int D, bool NV>
-static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                             const AttnParams& p, cudaStream_t stream) {
   const bool dbg = p.dbg_codes != nullptr;
   if (p.pnq == 2) {
     if constexpr (NV) return cudaErrorInvalidValue;    // the exp-free rule is MXFP4 only
-    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, p, stream)
-                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, p, stream);
+    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
+                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
   }
-  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, p, stream)
-                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, p, stream);
-  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, p, stream)
-             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, p, stream);
+  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
+                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
+  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
+             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
 }
 
 template <int D>
-static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                             const AttnParams& p, cudaStream_t stream) {
-  return p.mode == kModeNvfp4 ? launch_f<D, true>(tmQ, tmK, tmV, p, stream)
-                              : launch_f<D, false>(tmQ, tmK, tmV, p, stream);
+  return p.mode == kModeNvfp4 ? launch_f<D, true>(tmQ, tmK, tmV, tmO, p, stream)
+                              : launch_f<D, false>(tmQ, tmK, tmV, tmO, p, stream);
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                             const CUtensorMap& tmO,
                              const AttnParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, p, stream);
-  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, p, stream);
+  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, tmO, p, stream);
+  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, tmO, p, stream);
   return cudaErrorInvalidValue;
 }
 
