@@ -234,8 +234,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
 template <int D, int PM, bool DBG, bool NV>
 __global__ void __launch_bounds__(kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                      const AttnParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   static_assert(PM >= 0 && PM <= 2 && !(NV && PM == 2), "P~ rule");
   static_assert(offsetof(Smem<D>, p) % 1024 == 0 && sizeof(Smem<D>::p[0]) == 4 * 4096,
                 "the output stage needs four 1024-aligned 4 KB quarters per query tile");
@@ -733,12 +732,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_wait_ld();
       }
       const float inv_l = 1.f / l;
-      // The normalised rows leave through shared memory and tiled TMA stores, so that the global
-      // writes are whole lines: each warp stages a 32-row x 128-byte chunk (32 fp32 or 64 bf16
-      // columns) in its quarter of its query tile's P~ buffers, which no product reads any more
-      // once the last P~V product has completed. 128-byte swizzle: the 16-byte piece j of row r
-      // sits at position j ^ (r & 7), so the eight stores of a warp cover all banks. The tensor
-      // map is [B*Hq][N][D]: rows past N are clipped by the copy.
+      // The normalised rows leave through shared memory so that the global writes are whole lines:
+      // each warp stages a 32-row x 128-byte chunk (32 fp32 or 64 bf16 columns, its threads' rows)
+      // in its quarter of its query tile's P~ buffers, which no product reads any more once the
+      // last P~V product has completed, then reads it back four rows per instruction (eight
+      // lanes per 128-byte line). 128-byte swizzle: the 16-byte piece j of row r sits at position
+      // j ^ (r & 7), so that neither the row-wise writes nor the line-wise reads conflict on banks.
       uint8_t* stage = s.p[x][0] + quarter * 4096;
       const uint32_t row_addr = smem_u32(stage) + static_cast<uint32_t>(lane) * 128u;
       const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
@@ -749,10 +748,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(o_col + cc * 32, raw);
         tc_wait_ld();
         const bool half2 = p.out_bf16 && (cc & 1);        // bf16: second half of a 128-byte row
-        if (cc > 0 && !half2) {                           // the previous chunk's copy has read the stage
-          if (lane == 0) bulk_wait_group_read0();
-          __syncwarp();
-        }
         if (p.out_bf16) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -775,17 +770,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                          __float_as_uint(__uint_as_float(raw[4 * v + 3]) * inv_l));
         }
         if (!p.out_bf16 || half2) {
-          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            if (y0 < p.N) tma_store_3d(&tmO, stage, p.out_bf16 ? (cc >> 1) * 64 : cc * 32, y0, bh_q);
-            bulk_commit_group();
+          const int es = p.out_bf16 ? 2 : 4;
+          const int pc = lane & 7;
+          uint8_t* gbase = static_cast<uint8_t*>(p.out) + static_cast<size_t>(bh_q) * p.N * D * es +
+                           (p.out_bf16 ? (cc >> 1) * 128 : cc * 128) + pc * 16;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + (lane >> 3);
+            const uint4 val = ld_shared_v4(smem_u32(stage) + rr * 128 + ((pc ^ (rr & 7)) << 4));
+            if (y0 + rr < p.N) *reinterpret_cast<uint4*>(gbase + static_cast<size_t>(y0 + rr) * D * es) = val;
           }
+          __syncwarp();     // the stage is read before the next chunk overwrites it
         }
       }
-      // the stage must stay valid until the copies have read it
-      if (lane == 0) bulk_wait_group_read0();
-      __syncwarp();
     }
     tc_fence_before();
   }
@@ -798,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int PM, bool DBG, bool NV>
-static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
+static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
   // the softmax warpgroups' register increase is served from the block's launch allocation: a
@@ -816,37 +814,36 @@ static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
   if (e != cudaSuccess) return e;
   const unsigned n_units = static_cast<unsigned>((p.Npad / kBM + 1) / 2);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * n_units;
-  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, tmO, p);
+  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
 template <int D, bool NV>
-static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
+static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const bool dbg = p.dbg_codes != nullptr;
   if (p.pnq == 2) {
     if constexpr (NV) return cudaErrorInvalidValue;    // the exp-free rule is MXFP4 only
-    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
-                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
+    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, p, stream)
+                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, p, stream);
   }
-  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
-                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
-  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, tmO, p, stream)
-             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, tmO, p, stream);
+  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, p, stream)
+                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, p, stream);
+  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, p, stream)
+             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, p, stream);
 }
 
 template <int D>
-static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
+static cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
-  return p.mode == kModeNvfp4 ? launch_f<D, true>(tmQ, tmK, tmV, tmO, p, stream)
-                              : launch_f<D, false>(tmQ, tmK, tmV, tmO, p, stream);
+  return p.mode == kModeNvfp4 ? launch_f<D, true>(tmQ, tmK, tmV, p, stream)
+                              : launch_f<D, false>(tmQ, tmK, tmV, p, stream);
 }
 
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                             const CUtensorMap& tmO,
                              const AttnParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, tmO, p, stream);
-  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, tmO, p, stream);
+  if (d == 128) return launch_d<128>(tmQ, tmK, tmV, p, stream);
+  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, p, stream);
   return cudaErrorInvalidValue;
 }
 

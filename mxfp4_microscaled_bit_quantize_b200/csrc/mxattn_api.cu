@@ -98,23 +98,6 @@ bool make_map_typed(CUtensorMap* m, CUtensorMapDataType dtype, const void* base,
   return r == CUDA_SUCCESS;
 }
 
-// 3-D tensor map of the attention output [heads][N][d] (fp32 or bf16): box of 32 rows x 128 bytes
-// of one head, 128-byte swizzle; the copy clips rows past N, so a ragged last query tile stays
-// inside its own head.
-bool make_out_map(CUtensorMap* m, void* out, int bf16, uint64_t heads, uint64_t n, uint64_t d) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const uint64_t es = bf16 ? 2 : 4;
-  cuuint64_t dims[3] = {d, n, heads};
-  cuuint64_t strides[2] = {d * es, n * d * es};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 mxattn_status prepare_impl(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                            int scale_mode, void* ws, size_t ws_bytes, cudaStream_t st, const WsLayout& L) {
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -208,14 +191,13 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
                           int dbg_bh, int dbg_r0, int dbg_r1, uint8_t* p_codes, uint8_t* p_scales,
                           unsigned int* status = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   const uint64_t rph = static_cast<uint64_t>(src.rows_per_head);
   if (!make_map(&tq, src.qc, d / 2, static_cast<uint64_t>(B) * Hq * rph, d / 2, kTile, qk_swz) ||
       !make_map(&tk, src.kc, d / 2, static_cast<uint64_t>(B) * Hkv * rph, d / 2, kKvTile, qk_swz) ||
       !make_map(&tv, src.vc, src.v_row_bytes, static_cast<uint64_t>(B) * Hkv * d, kKvTile / 2, d,
-                CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_out_map(&to, out, out_dtype == MXATTN_OUT_BF16, static_cast<uint64_t>(B) * Hq, N, d))
+                CU_TENSOR_MAP_SWIZZLE_64B))
     return MXATTN_ERR_CUDA;
   AttnParams p{};
   p.qsf = w + L.qs;
@@ -239,7 +221,7 @@ mxattn_status attend_impl(void* out, int B, int Hq, int Hkv, int N, int d, int c
   p.dbg_bh = dbg_bh;
   p.dbg_r0 = dbg_r0;
   p.dbg_r1 = dbg_r1;
-  return launch_attention(tq, tk, tv, to, p, d, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+  return launch_attention(tq, tk, tv, p, d, st) == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
 mxattn_status check_forward_args(const void* q, const void* k, const void* v, const void* out, int B, int Hq,

@@ -109,10 +109,7 @@ struct AttnParams {
   int dbg_bh, dbg_r0, dbg_r1;
 };
 
-// tmO: the output [B*Hq][N][d] (fp32 or bf16) as a 3-D map with a 32-row x 128-byte box and
-// 128-byte swizzle; the kernel writes it with tiled TMA stores.
 cudaError_t launch_attention(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                             const CUtensorMap& tmO,
                              const AttnParams& p, int d, cudaStream_t stream);
 
 // Block-scaled MXFP4 GEMM C[M, N] = dq(A) dq(B)^T; A, B codes are read through tensor maps, their
