@@ -26,7 +26,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "video_dit"
-OTHER_CONFIGS = ("video_dit_long", "llm_gqa")   # also timed, attention per step (UOS + PNQ)
+# also timed, quantizers + attention per step, PNQ: (key, workload, scale mode); the long video DiT
+# runs under both MXFP4 scale rules, UOS against the OCP baseline
+OTHER_CONFIGS = (("video_dit_long", "video_dit_long", "uos"), ("video_dit_long_ocp", "video_dit_long", "ocp"),
+                 ("llm_gqa", "llm_gqa", "uos"))
 METRIC = "MXFP4 attention fwd TFLOP/s (video-DiT 1x40x32760x128, UOS+PNQ)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 FP4_PER_BF16 = 4.0          # nominal dense ratio: 9 PFLOP/s fp4 vs 2.25 PFLOP/s bf16
@@ -436,8 +439,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     # the other full-size attention workloads: the long video DiT and the causal GQA prefill
     # (quantizers + attention kernel per step, timed per phase as in the main loop)
     other = {}
-    for name in OTHER_CONFIGS:
-        ocfg = synthetic.ATTN_CONFIGS[name]
+    for name, wl, scale in OTHER_CONFIGS:
+        ocfg = synthetic.ATTN_CONFIGS[wl]
+        o_mode = {"uos": api.SCALE_UOS, "ocp": api.SCALE_OCP}[scale]
         oq, ok_, ov = (t.to(dev) for t in synthetic.attn_inputs(ocfg))
         o_ws = api.alloc_workspace(ocfg.B, ocfg.Hq, ocfg.Hkv, ocfg.N, ocfg.d, dev)
         o_out = torch.empty((ocfg.B, ocfg.Hq, ocfg.N, ocfg.d), dtype=torch.float32, device=dev)
@@ -445,10 +449,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         def o_step(e=None):
             if e is not None:
                 e[0].record(stream)
-            api.mxattn_forward_prepare(oq, ok_, ov, api.SCALE_UOS, o_ws)
+            api.mxattn_forward_prepare(oq, ok_, ov, o_mode, o_ws)
             if e is not None:
                 e[1].record(stream)
-            api.mxattn_forward_attend(o_out, ocfg.B, ocfg.Hq, ocfg.Hkv, ocfg.N, ocfg.d, ocfg.causal, api.SCALE_UOS,
+            api.mxattn_forward_attend(o_out, ocfg.B, ocfg.Hq, ocfg.Hkv, ocfg.N, ocfg.d, ocfg.causal, o_mode,
                                       True, o_ws)
             if e is not None:
                 e[2].record(stream)
@@ -504,7 +508,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     quant_alone_ms, xq0_numel = time_quantizer_rotating(dev, stream, barrier, iters=50)
 
     # max over ranks
-    other_ms = [x for name in OTHER_CONFIGS for x in other[name][1:]]
+    other_ms = [x for name, _, _ in OTHER_CONFIGS for x in other[name][1:]]
     (step_ms, attn_ms, quant_ms, e2e_ms, copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms,
      nv_attn_ms, efq_attn_ms, *other_ms) = reduce_max_over_ranks([total_ms / args.steps, attn_ms, quant_ms, e2e_ms,
                                                      copy_ms, quant_alone_ms, fq_ms, gemm_ms, gemm_nv_ms, nv_attn_ms,
@@ -560,13 +564,13 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "forward_quantized": {"ms": fq_ms, "tflops": flops / (fq_ms * 1e-3) / 1e12,
                               "note": "mxattn_forward_quantized on pre-quantized Q/K/V: scale repack + kernel"},
         "other_configs": {
-            name: {"workload": other[name][0].describe(), "attn_ms": other_ms[2 * i],
+            name: {"workload": other[name][0].describe(), "scale_mode": scale.upper(), "attn_ms": other_ms[2 * i],
                    "tflops": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12,
                    "frac": other[name][0].flops / (other_ms[2 * i] * 1e-3) / 1e12 / fp4_peak,
                    "step_ms": other_ms[2 * i + 1],
                    "step_tflops": other[name][0].flops / (other_ms[2 * i + 1] * 1e-3) / 1e12,
                    "traffic": profile_traffic(f"attn_fwd_{name}.json", sources_hash(ATTN_SOURCES))}
-            for i, name in enumerate(OTHER_CONFIGS)},
+            for i, (name, _, scale) in enumerate(OTHER_CONFIGS)},
         "gemm": {"workload": f"mxattn_gemm W4A4 {gm}x{gn}x{gk}, bf16 out", "ms": gemm_ms,
                  "tflops": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12,
                  "frac": 2.0 * gm * gn * gk / (gemm_ms * 1e-3) / 1e12 / fp4_peak,
@@ -662,7 +666,7 @@ def main():
     ap.add_argument("--mode", choices=["full", "attention", "quantizer", "gemm"], default="full",
                     help="attention / quantizer: time only that part (small cases for profiling)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling only)")
-    ap.add_argument("--workload", choices=[WORKLOAD, *OTHER_CONFIGS], default=WORKLOAD,
+    ap.add_argument("--workload", choices=[WORKLOAD, *sorted({wl for _, wl, _ in OTHER_CONFIGS})], default=WORKLOAD,
                     help="the attention workload of --mode attention (profiling only)")
     ap.add_argument("--p-rule", choices=["conventional", "pnq", "efq"], default="pnq",
                     help="the P~ rule of --mode attention (profiling only)")
