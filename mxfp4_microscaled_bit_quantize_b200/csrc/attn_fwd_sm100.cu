@@ -398,12 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; ok && t < n_kv_max; ++t) {
       const int st = t % NS;
       const int pb = t & 1;
-      if (t >= n_own) {
-        // no product of this query tile reads key tile t: count this issuer's release of the stage
-        if (leader) mbar_arrive(&s.bar_kv_empty[st]);
-        __syncwarp();
-        continue;
-      }
+      // no product of this query tile reads key tile t: the other issuer releases the stage for
+      // both (an issuer that arrived here on its own could run ahead and arrive twice on one phase)
+      if (t >= n_own) continue;
       ok = warp_wait(&s.bar_p_full[x][pb], (t >> 1) & 1, abort_flag, p.status, kStatusTimeoutP);
       if (!ok) break;
       // The V scale atoms of key tile t are copied by its first product: PV(A, t), or PV(B, t) when
@@ -446,8 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(&s.bar_pv_done[x][pb]);
         // this issuer's release of the stage: the S products that read its K tile were complete
-        // before this product's softmax could read S(x, t)
+        // before this product's softmax could read S(x, t). When the other tile has no product at
+        // key tile t, the second arrival is made here too; the phase still completes only with
+        // the commit.
         tc_commit(&s.bar_kv_empty[st]);
+        if (t >= n_other) mbar_arrive(&s.bar_kv_empty[st]);
       }
       __syncwarp();
     }

@@ -96,6 +96,30 @@ def test_shapes_exp_free(dev, N, d, causal):
     _run_and_check(dev, q, k, v, causal, mx.SCALE_UOS, oa.P_EFQ, [(0, 0), (0, 3)])
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_odd_tile_count_long_rows(dev, d, causal):
+    """An odd number of query tiles (the last tile pair of each head has no tile B, so one P~V
+    issuer has no product at any key tile) with more key tiles than pipeline stages (6 for
+    d = 128, 8 for d = 64), and more tile pairs than SMs."""
+    N = 1100                                       # 9 query tiles, 9 key tiles
+    q, k, v = _rand_qkv(1, 72, 18, N, d, seed=2000 + d + causal, qk_scale=1.5)
+    _run_and_check(dev, q, k, v, causal, mx.SCALE_UOS, True, [(0, 0), (0, 37), (0, 71)])
+
+
+@pytest.mark.parametrize("mode,pnq", [(mx.SCALE_OCP, oa.P_EFQ), (mx.SCALE_UOS, False)])
+def test_odd_tile_count_other_rules(dev, mode, pnq):
+    q, k, v = _rand_qkv(2, 40, 8, 1100, 128, seed=2100 + int(pnq), qk_scale=1.5)
+    _run_and_check(dev, q, k, v, True, mode, pnq, [(0, 5), (1, 39)])
+
+
+def test_bf16_output_ragged_odd_tiles(dev):
+    q, k, v = _rand_qkv(1, 64, 16, 1100, 64, seed=2200)
+    o32 = api.mxattn_forward(q.to(dev), k.to(dev), v.to(dev), causal=True)
+    o16 = api.mxattn_forward(q.to(dev), k.to(dev), v.to(dev), causal=True, out_dtype=torch.bfloat16)
+    assert torch.equal(o16.float(), o32.bfloat16().float())
+
+
 def test_gqa_and_batches(dev):
     q, k, v = _rand_qkv(2, 8, 2, 200, 128, seed=11)
     _run_and_check(dev, q, k, v, True, mx.SCALE_UOS, True, [(0, 0), (0, 5), (1, 3), (1, 7)])
