@@ -170,13 +170,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, code));
 }
 
-// E8M0 byte of a P~ block maximum amax in [0, 1] (the running max bounds every P~ by 1): the OCP
-// exponent floor(log2 amax) - 2 read off the fp32 exponent field, plus one under UOS when the
-// significand exceeds 1.8125; byte 0 for amax = 0 and for every amax whose exponent would fall
-// below -127 (subnormal or tiny maxima), as the general rule's clamp gives.
-__device__ __forceinline__ uint32_t p_scale_byte(float amax, int mode) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int byte = static_cast<int>(bits >> 23) - 2 + ((mode == 1 && (bits & 0x7FFFFFu) > 0x680000u) ? 1 : 0);
+// E8M0 byte of a P~ block maximum amax = 2^d in [0, 1] (the running max bounds every P~ by 1),
+// read off d <= 0 itself, with no exponential: the OCP exponent floor(log2 amax) - 2 = floor(d) - 2,
+// plus one under UOS when the significand 2^f, f = d - floor(d), exceeds 1.8125, i.e. when
+// f > log2 1.8125 (0x1.b74948p-1 in fp32, whose 2^f is just below 1.8125). floor(d) comes from one
+// round-down add of 1.5 * 2^23 (the sum's low mantissa bits then hold it) and f is exact. Every d
+// below -126, d = -inf (an all-masked block) included, gives byte 0, as the general rule's clamp
+// does for subnormal and zero maxima.
+__device__ __forceinline__ uint32_t p_scale_byte_log2(float d, int mode) {
+  constexpr float kMagic = 12582912.0f;                   // 1.5 * 2^23
+  constexpr float kLog2UosLimit = 0x1.b74948p-1f;         // log2(1.8125) rounded to fp32
+  const float dc = fmaxf(d, -160.f);
+  const float t = __fadd_rd(dc, kMagic);                  // floor(dc) + 1.5 * 2^23, exactly
+  const int e = __float_as_int(t) - 0x4B400000;           // floor(dc)
+  const float f = dc - (t - kMagic);
+  const int byte = e + 125 + ((mode == 1 && f > kLog2UosLimit) ? 1 : 0);
   return static_cast<uint32_t>(max(byte, 0));
 }
 
@@ -588,15 +596,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bb = 1; bb < kNPB; ++bb) tmax = fmaxf(tmax, bmax[bb]);
       const float m_new = fmaxf(m, tmax);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
+      // the history factor alpha = 2^((m - m') c) only where some row of the warp saw its max move
+      // (elsewhere it is 1); it is read by the rescale below and by the conventional row sum
+      const bool moved = __any_sync(0xffffffffu, m_new > m);
+      float alpha = 1.f;
+      if (moved) alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
 
       uint32_t sbytes[kNPB / 4];
       float nb[kNPB], bscale[kNPB];
 #pragma unroll
       for (int bb = 0; bb < kNPB; ++bb) {
-        const float amax = ex2_approx((bmax[bb] - m_use) * c);     // 0 for an all-masked block
         uint32_t byte;
         if constexpr (NV) {
+          const float amax = ex2_approx((bmax[bb] - m_use) * c);   // 0 for an all-masked block
           // s = E4M3(amax / 6) with both quotients correctly rounded. s = 0 (amax <= 6 * 2^-10):
           // y = P~ itself (every value below the 0.25 rounding threshold, so the codes are 0 as
           // the format wants) and the unquantized row sum still counts the block with weight 1
@@ -605,7 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           bscale[bb] = sb > 0.f ? sb : 1.f;
           nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
         } else {
-          byte = p_scale_byte(amax, p.mode);
+          // the byte of amax = 2^((bmax - m') c) straight from the exponent (no MUFU on this path)
+          byte = p_scale_byte_log2((bmax[bb] - m_use) * c, p.mode);
           // 127 - byte as a float without a conversion: it sits in the low mantissa bits of 2^23
           const float neg_e = __uint_as_float(0x4B000000u + (127u - byte)) - 8388608.0f;
           nb[bb] = fmaf(-m_use, c, neg_e);
@@ -686,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // history rescale of O and L (only when some row of this warp saw its max move); O may only
       // be touched once the product of key tile t-1 has landed in it
-      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (t > 0 && moved) {
         ok = warp_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
         if (!ok) break;
         tc_fence_after();
