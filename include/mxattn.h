@@ -264,9 +264,8 @@ mxattn_status mxattn_forward_debug(const void* q, const void* k, const void* v, 
  *   - All calls on a device share the array: calls whose kernels overlap on the GPU race, so
  *     serialise them (one stream, or explicit ordering). The status word is cleared at the
  *     start of each call. A device-side wait timeout is recorded only in the shared array,
- *     which no caller can read: the call has already returned MXATTN_OK and `out` is then
- *     unspecified. Callers that must detect timeouts use mxattn_forward with their own
- *     workspace and mxattn_check_status.
+ *     which no caller can read directly: the call has already returned MXATTN_OK and `out` is
+ *     then unspecified. mxattn_check_status_noalloc reads (and clears) that word.
  */
 #define MXATTN_NOALLOC_MAX_WORKSPACE ((size_t)16 << 20)
 mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq,
@@ -279,6 +278,14 @@ mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v
  * raw code goes to *detail when detail != NULL), MXATTN_ERR_CUDA on a CUDA error, else MXATTN_OK.
  */
 mxattn_status mxattn_check_status(void* workspace, void* stream, unsigned int* detail);
+
+/*
+ * mxattn_check_status_noalloc -- mxattn_check_status on the static array that
+ * mxattn_forward_noalloc uses as its workspace, in the current context: synchronises `stream`,
+ * reads and clears the status word the last mxattn_forward_noalloc calls wrote. Same returns as
+ * mxattn_check_status. Like the forward call, it allocates nothing.
+ */
+mxattn_status mxattn_check_status_noalloc(void* stream, unsigned int* detail);
 
 /* Static string for a status code. */
 const char* mxattn_status_string(int status);

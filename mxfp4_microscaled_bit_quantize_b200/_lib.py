@@ -34,6 +34,7 @@ SIGNATURES = {
     "mxattn_gemm_nvfp4_workspace_size": (_c_size, [_c_i64] * 3),
     "mxattn_gemm_nvfp4": (_c_int, [_u8p] * 4 + [_vp] + [_c_i64] * 3 + [_c_int, _vp, _c_size, _vp]),
     "mxattn_check_status": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_uint)]),
+    "mxattn_check_status_noalloc": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint)]),
     "mxattn_status_string": (ctypes.c_char_p, [_c_int]),
     "mxattn_version": (_c_int, []),
 }

@@ -373,7 +373,7 @@ mxattn_status mxattn_quantize_nvfp4(const void* x, int64_t rows, int64_t cols, u
 }
 
 
-int mxattn_version(void) { return 101; }
+int mxattn_version(void) { return 102; }
 
 const char* mxattn_status_string(int status) {
   switch (status) {

@@ -56,3 +56,10 @@ extern "C" mxattn_status mxattn_forward_noalloc(const void* q, const void* k, co
   return mxattn_forward(q, k, v, out, B, Hq, Hkv, N, d, causal, scale_mode, pnq, out_dtype, scratch,
                         kNoAllocScratchBytes, stream);
 }
+
+extern "C" mxattn_status mxattn_check_status_noalloc(void* stream, unsigned int* detail) {
+  void* scratch = nullptr;
+  const mxattn_status s = scratch_for_current_context(&scratch);
+  if (s != MXATTN_OK) return s;
+  return mxattn_check_status(scratch, stream, detail);
+}

@@ -81,3 +81,17 @@ def test_noalloc_rejects_like_forward(lib, shape, expected):
     ws_bytes = min(lib.mxattn_forward_workspace_size(B, Hq, Hkv, N, d), MAX_WORKSPACE) or MAX_WORKSPACE
     r_fwd = lib.mxattn_forward(fake, fake, fake, fake, B, Hq, Hkv, N, d, 0, 1, 1, 0, fake, ws_bytes, None)
     assert r_fwd == expected
+
+
+def test_noalloc_status_word_reads_clean(lib):
+    """After good noalloc calls the static array's status word reads 0, and reading clears it."""
+    dev = torch.device("cuda:0")
+    cfg = synthetic.ATTN_CONFIGS["tiny"]
+    q, k, v = (t.to(dev) for t in synthetic.attn_inputs(cfg))
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    assert _noalloc(lib, q, k, v, out, False, mx.SCALE_UOS, True) == 0
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    for _ in range(2):
+        detail = ctypes.c_uint(123)
+        assert lib.mxattn_check_status_noalloc(stream, ctypes.byref(detail)) == 0
+        assert detail.value == 0
