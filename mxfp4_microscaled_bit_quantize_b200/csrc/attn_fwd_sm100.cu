@@ -609,10 +609,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t byte;
         if constexpr (NV) {
           const float amax = ex2_approx((bmax[bb] - m_use) * c);   // 0 for an all-masked block
-          // s = E4M3(amax / 6) with both quotients correctly rounded. s = 0 (amax <= 6 * 2^-10):
-          // y = P~ itself (every value below the 0.25 rounding threshold, so the codes are 0 as
-          // the format wants) and the unquantized row sum still counts the block with weight 1
-          byte = e4m3_byte(__fdiv_rn(amax, 6.0f));
+          // s = E4M3(amax / 6), the quotient as amax times fp32(1/6): within one ulp of the
+          // correctly rounded quotient, so the E4M3 rounding can only differ where the quotient
+          // lies within an ulp of one of its midpoints (amax itself comes from ex2.approx). s = 0
+          // (amax <= 6 * 2^-10): y = P~ itself (every value below the 0.25 rounding threshold,
+          // so the codes are 0 as the format wants) and the unquantized row sum still counts the
+          // block with weight 1
+          byte = e4m3_byte(amax * (1.0f / 6.0f));
           const float sb = e4m3_value(byte);
           bscale[bb] = sb > 0.f ? sb : 1.f;
           nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
