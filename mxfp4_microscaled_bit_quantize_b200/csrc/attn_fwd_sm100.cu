@@ -60,7 +60,7 @@ namespace mxattn {
 
 constexpr int kBM = 128;          // query rows per Q tile (the MMA's M)
 constexpr int kBN = kKvTile;      // keys per KV tile (128)
-constexpr int kThreads = 384;     // warpgroup 0: producer, MMA, 2 idle; warpgroups 1, 2: softmax A, B
+constexpr int kThreads = 384;     // warpgroup 0: TMA, S issuer, two P~V issuers; warpgroups 1, 2: softmax A, B
 // Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for 384
 // threads); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to kSoftmaxRegs.
 // The three shares add up to exactly the launch total, which the host checks before launching.
@@ -75,7 +75,7 @@ constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 
 //   ones        kColSf1 + 4 X (one copy per P~V issuer)
 // tcgen05.cp into columns an earlier MMA still reads is not ordered behind that MMA; the K, V and
 // P~ sets alternate by tile parity, and the set written for tile t was last read by a product of
-// tile t - 2, which the issuing thread has seen complete by then (see the MMA issuer).
+// tile t - 2, which the copying thread has seen complete by then (see the S and P~V issuers).
 constexpr uint32_t kColSfQ = 416, kColSfK = 432, kColSfV = 448, kColSfP = 464, kColSf1 = 496;   // + 4 x
 constexpr int kOnesRows = 16;     // N of the row-sum MMA: row 0 all ones, rows 1..15 zero
 constexpr int kPRowBytes = kBN / 2;                  // 64 bytes of codes per P~ / V^T row
@@ -321,9 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
    regs_dec<kCtlRegs>();
-   // Two issuing warps on different SM sub-partitions share the tcgen05 work: warp 1 the S
-   // products (the latency-critical hand-overs of the S buffer), warp 0 the TMA loads and the
-   // P~V and row-sum products. Each waits on the barriers that gate its own products; the
+   // Four control warps, one per SM sub-partition: warp 2 the TMA loads, warp 1 the S products
+   // (the latency-critical hand-overs of the S buffer), warps 0 and 3 the P~V and row-sum
+   // products of tiles A and B. Each waits on the barriers that gate its own work; the
    // scale-atom sets stay safe as argued beside each copy below.
    const uint64_t sf_desc_base = smem_desc(0, 0, 128, kLayoutNone);
    auto sf_desc = [&](const void* ptr) { return sf_desc_base | ((smem_u32(ptr) >> 4) & 0x3FFFu); };
