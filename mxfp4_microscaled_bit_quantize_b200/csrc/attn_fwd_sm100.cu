@@ -707,10 +707,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         {
+          // O and (PNQ) L in one batch of loads behind one wait, then one batch of stores
           uint32_t raw[D];
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc)
             tmem_ld32(o_col + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
+          const uint32_t lv = PNQ ? tmem_ld1(l_col) : 0u;
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < D; i += 2) {
@@ -722,11 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc)
             tmem_st32(o_col + cc * 32, *reinterpret_cast<const uint32_t(*)[32]>(raw + 32 * cc));
-        }
-        if (PNQ) {
-          const uint32_t lv = tmem_ld1(l_col);
-          tc_wait_ld();
-          tmem_st1(l_col, __float_as_uint(__uint_as_float(lv) * alpha));
+          if (PNQ) tmem_st1(l_col, __float_as_uint(__uint_as_float(lv) * alpha));
         }
         tc_wait_st();
       }
