@@ -21,8 +21,8 @@
 // S(A, t+1), ... . Their softmax warps therefore run half a step apart, and on every SM
 // sub-partition one tile's serial work (S load, maxima, scale selection, stores, rescale) overlaps
 // the other tile's exponentials on the MUFU.
-// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 104 registers
-// per thread and each softmax warpgroup 200):
+// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 88 registers
+// per thread and each softmax warpgroup 208):
 //   warp 2     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
 //              an NSTAGE-deep shared-memory ring (mbarrier complete_tx).
 //   warp 1     TMEM owner and S issuer (one thread): copies the Q and K scale atoms and issues
@@ -64,7 +64,7 @@ constexpr int kThreads = 384;     // warpgroup 0: TMA, S issuer, two P~V issuers
 // Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for 384
 // threads); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to kSoftmaxRegs.
 // The three shares add up to exactly the launch total, which the host checks before launching.
-constexpr int kLaunchRegs = 168, kCtlRegs = 104, kSoftmaxRegs = 200;
+constexpr int kLaunchRegs = 168, kCtlRegs = 88, kSoftmaxRegs = 208;
 static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 X, L_X at kColL + 16 X
