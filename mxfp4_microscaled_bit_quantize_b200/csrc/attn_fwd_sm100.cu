@@ -60,12 +60,26 @@ namespace mxattn {
 
 constexpr int kBM = 128;          // query rows per Q tile (the MMA's M)
 constexpr int kBN = kKvTile;      // keys per KV tile (128)
-constexpr int kThreads = 384;     // warpgroup 0: TMA, S issuer, two P~V issuers; warpgroups 1, 2: softmax A, B
-// Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for 384
-// threads); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to kSoftmaxRegs.
-// The three shares add up to exactly the launch total, which the host checks before launching.
-constexpr int kLaunchRegs = 168, kCtlRegs = 88, kSoftmaxRegs = 208;
-static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs == kThreads * kLaunchRegs, "register split");
+// Two softmax layouts (the kernel's WS parameter, softmax warps per query tile):
+//   WS = 4: one thread per query row, 384 threads (warpgroup 0 control, warpgroups 1-2 softmax).
+//   WS = 8: two threads per query row (each a 64-key half of every key tile), 640 threads
+//           (warpgroup 0 control, warpgroups 1-4 softmax): twice the warps on each SM
+//           sub-partition to cover the softmax chain's waits, in half the registers per thread.
+// Register split (per thread): the block is launched with kLaunchRegs (the ptxas limit for its
+// thread count); warpgroup 0 gives back down to kCtlRegs, the softmax warpgroups grow to
+// kSoftmaxRegs. The shares add up to exactly the launch total, which the host checks before
+// launching.
+template <int WS> struct Layout;
+template <> struct Layout<4> {
+  static constexpr int kThreads = 384, kLaunchRegs = 168, kCtlRegs = 88, kSoftmaxRegs = 208;
+};
+template <> struct Layout<8> {
+  static constexpr int kThreads = 640, kLaunchRegs = 96, kCtlRegs = 64, kSoftmaxRegs = 104;
+};
+static_assert(128 * Layout<4>::kCtlRegs + 256 * Layout<4>::kSoftmaxRegs == Layout<4>::kThreads * Layout<4>::kLaunchRegs,
+              "register split");
+static_assert(128 * Layout<8>::kCtlRegs + 512 * Layout<8>::kSoftmaxRegs == Layout<8>::kThreads * Layout<8>::kLaunchRegs,
+              "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColL = 384;   // O_X at kColO + 128 X, L_X at kColL + 16 X
 // Scale atoms, 4 columns each (NVFP4 needs two per operand tile, MXFP4 one):
@@ -193,7 +207,8 @@ __device__ __forceinline__ uint32_t p_scale_byte_log2(float d, int mode) {
 // the tcgen05 issue work spread over all four SM sub-partitions the softmax warps set the pace and
 // the MUFU (16 results per clock per SM) is their busiest unit; measured on the video-DiT workload,
 // 4, 5, 6 and 7 of 16 pairs gave +2%, +7%, +3% and +1% over none.
-constexpr int kPolyPairs = 5;
+constexpr int kPolyPairs8 = 5, kPolyPairs16 = 3;   // one / two threads per row (WS = 4 / 8)
+template <int kPolyPairs>
 __host__ __device__ constexpr bool poly_pair(int pair) {
   return ((pair + 1) * kPolyPairs) / 16 > (pair * kPolyPairs) / 16;
 }
@@ -237,13 +252,27 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
+// One thread's half of a row of D TMEM columns (D / 2 per thread, the halves 64 or 32 apart).
+template <int D>
+__device__ __forceinline__ void tmem_ld16x2_h(uint32_t taddr, uint32_t (&r)[D / 2]) {
+  if constexpr (D == 128) tmem_ld16x2_64<64>(taddr, r);
+  else tmem_ld16x2_32<32>(taddr, r);
+}
+template <int D>
+__device__ __forceinline__ void tmem_st16x2_h(uint32_t taddr, const uint32_t (&r)[D / 2]) {
+  if constexpr (D == 128) tmem_st16x2_64<64>(taddr, r);
+  else tmem_st16x2_32<32>(taddr, r);
+}
+
 // NV = false: MXFP4 (blocks of 32, UE8M0, OCP or UOS exponent). NV = true: the NVFP4 comparison
 // format for Q, K, V and P~ (blocks of 16, E4M3 scale = RNE(amax / 6)).
-template <int D, int PM, bool DBG, bool NV>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int PM, bool DBG, bool NV, int WS>
+__global__ void __launch_bounds__(Layout<WS>::kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   static_assert(PM >= 0 && PM <= 2 && !(NV && PM == 2), "P~ rule");
+  static_assert(WS == 4 || WS == 8, "softmax layout");
+  constexpr int kCtlRegs = Layout<WS>::kCtlRegs, kSoftmaxRegs = Layout<WS>::kSoftmaxRegs;
   static_assert(offsetof(Smem<D>, p) % 1024 == 0 && sizeof(Smem<D>::p[0]) == 4 * 4096,
                 "the output stage needs four 1024-aligned 4 KB quarters per query tile");
   constexpr bool PNQ = PM != 0;     // the row sum is the ones-operand product of the quantized P~
@@ -299,11 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s.bar_s_full[x], 1);
       for (int i = 0; i < 2; ++i) {
-        mbar_init(&s.bar_p_full[x][i], 4);      // one arrival per softmax warp of the tile
+        mbar_init(&s.bar_p_full[x][i], WS);     // one arrival per softmax warp of the tile
         mbar_init(&s.bar_pv_done[x][i], 1);
       }
     }
-    mbar_init(&s.bar_s_empty, 4);
+    mbar_init(&s.bar_s_empty, WS);
     for (int i = 0; i < 3; ++i) mbar_init(&s.bar_drain[i], 1);
     mbar_init(&s.bar_ones, 1);
     s.abort_flag = 0;
@@ -539,267 +568,559 @@ __global__ void __launch_bounds__(kThreads, 1)
    }
   } else {
     regs_inc<kSoftmaxRegs>();
-    // ============================ softmax warps ============================
-    const int x = (warp - 4) >> 2;                    // query tile: warps 4-7 A, 8-11 B
-    const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
-    const int r = quarter * 32 + lane;                // row inside the tile == TMEM lane
-    const int qt = x == 0 ? qt_x[0] : qt_x[1];
-    const int n_kv = x == 0 ? n_kv_x[0] : n_kv_x[1];
-    const int qrow = qt * kBM + r;
-    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t o_col = tmem + lane_addr + kColO + 128 * x;
-    const uint32_t l_col = tmem + lane_addr + kColL + 16 * x;
-    const float c = p.scale_log2;
-    constexpr int kPB = NV ? 16 : 32;                 // keys per P~ scale block
-    constexpr int kNPB = kBN / kPB;                   // scale blocks per row per tile
-    const float c27 = c * (2.f / 7.f);                // exp-free rule: (2 r + 2) / 7 = S c27 + b7
-    float m = -INFINITY;      // running max of the raw scores S
-    float l = 0.f;            // running row sum (pnq = 0)
-    bool ok = n_kv > 0;
-    const bool dbg = DBG && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
-    const uint32_t swz = (static_cast<uint32_t>(r) >> 1) & 3u;   // 64-byte swizzle of this row
-    const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
+    if constexpr (WS == 8) {
 
-    for (int t = 0; ok && t < n_kv; ++t) {
-      ok = warp_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8);
-      if (!ok) break;
-      tc_fence_after();
-      float sv[kBN];
-      {
-        uint32_t raw[kBN];
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc)
-          tmem_ld32(tmem + lane_addr + kColS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(raw[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.bar_s_empty);
+      // ============================ softmax warps ============================
+      // Two threads per query row: eight warps per tile, two per TMEM lane quarter (16 rows each).
+      // Thread (lane & 15) of a warp owns row r of its 16 and keys [64 kh, 64 kh + 64) of each key
+      // tile (kh = lane >> 4): the 16-lane, two-half TMEM load gives each half-warp the same lanes
+      // at columns 64 apart. The row max and the conventional row sum meet over one shuffle with
+      // the partner thread (lane ^ 16); block maxima, scale bytes and P~ codes stay thread-local.
+      const int sw = warp - 4;
+      const int x = sw >> 3;                            // query tile: warps 4-11 A, 12-19 B
+      const int hh = (sw >> 2) & 1;                     // which 16 rows of the lane quarter
+      const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
+      const int kh = lane >> 4;                         // key half of the tile (and of O's columns)
+      const int r0 = quarter * 32 + hh * 16;            // first row of this warp
+      const int r = r0 + (lane & 15);                   // row inside the tile == TMEM lane
+      const int qt = x == 0 ? qt_x[0] : qt_x[1];
+      const int n_kv = x == 0 ? n_kv_x[0] : n_kv_x[1];
+      const int qrow = qt * kBM + r;
+      const uint32_t lane_addr = static_cast<uint32_t>(r0) << 16;
+      const uint32_t o_col = tmem + lane_addr + kColO + 128 * x;
+      const uint32_t l_col = tmem + lane_addr + kColL + 16 * x;
+      const float c = p.scale_log2;
+      constexpr int kPB = NV ? 16 : 32;                 // keys per P~ scale block
+      constexpr int kNPB = kBN / kPB;                   // scale blocks per row per tile
+      constexpr int kNPBt = kNPB / 2;                   // ... of which this thread owns
+      constexpr int kHalf = kBN / 2;                    // keys per thread per tile
+      const float c27 = c * (2.f / 7.f);                // exp-free rule: (2 r + 2) / 7 = S c27 + b7
+      float m = -INFINITY;      // running max of the raw scores S
+      float l = 0.f;            // running row sum (pnq = 0), this thread's half
+      bool ok = n_kv > 0;
+      const bool dbg = DBG && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
+      const uint32_t swz = (static_cast<uint32_t>(r) >> 1) & 3u;   // 64-byte swizzle of this row
+      const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
 
-      // masking: keys beyond N, and keys after the query row when causal
-      const int key0 = t * kBN;
-      if (key0 + kBN > p.N || (p.causal && key0 + kBN - 1 > qt * kBM)) {
-        const int lim = (p.causal ? min(p.N, qrow + 1) : p.N) - key0;   // keys [key0, key0 + lim) count
-#pragma unroll
-        for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
-      }
-      // per block (32 keys for MXFP4, 16 for NVFP4): amax from the exact difference (1 for the
-      // block that holds the max), the block's scale byte, and the exponent bias nb of
-      // y = P~ / s = 2^(S c - m c - log2 s): one packed FMA per two elements and one ex2 each
-      float bmax[kNPB];
-#pragma unroll
-      for (int bb = 0; bb < kNPB; ++bb) bmax[bb] = NV ? block_max16(sv + bb * kPB) : block_max32(sv + bb * kPB);
-      float tmax = bmax[0];
-#pragma unroll
-      for (int bb = 1; bb < kNPB; ++bb) tmax = fmaxf(tmax, bmax[bb]);
-      const float m_new = fmaxf(m, tmax);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      // the history factor alpha = 2^((m - m') c) only where some row of the warp saw its max move
-      // (elsewhere it is 1); it is read by the rescale below and by the conventional row sum
-      const bool moved = __any_sync(0xffffffffu, m_new > m);
-      float alpha = 1.f;
-      if (moved) alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
-
-      uint32_t sbytes[kNPB / 4];
-      float nb[kNPB], bscale[kNPB];
-#pragma unroll
-      for (int bb = 0; bb < kNPB; ++bb) {
-        uint32_t byte;
-        if constexpr (NV) {
-          const float amax = ex2_approx((bmax[bb] - m_use) * c);   // 0 for an all-masked block
-          // s = E4M3(amax / 6), the quotient as amax times fp32(1/6): within one ulp of the
-          // correctly rounded quotient, so the E4M3 rounding can only differ where the quotient
-          // lies within an ulp of one of its midpoints (amax itself comes from ex2.approx). s = 0
-          // (amax <= 6 * 2^-10): y = P~ itself (every value below the 0.25 rounding threshold,
-          // so the codes are 0 as the format wants) and the unquantized row sum still counts the
-          // block with weight 1
-          byte = e4m3_byte(amax * (1.0f / 6.0f));
-          const float sb = e4m3_value(byte);
-          bscale[bb] = sb > 0.f ? sb : 1.f;
-          nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
-        } else {
-          // the byte of amax = 2^((bmax - m') c) straight from the exponent (no MUFU on this path)
-          byte = p_scale_byte_log2((bmax[bb] - m_use) * c, p.mode);
-          // 127 - byte as a float without a conversion: it sits in the low mantissa bits of 2^23
-          const float neg_e = __uint_as_float(0x4B000000u + (127u - byte)) - 8388608.0f;
-          nb[bb] = fmaf(-m_use, c, neg_e);
-          bscale[bb] = pow2_from_byte(byte);
-        }
-        if (bb % 4 == 0) sbytes[bb / 4] = 0;
-        sbytes[bb / 4] |= byte << (8 * (bb % 4));
-      }
-      // P~ buffer t&1: its last reader, the product of key tile t-2, completed before S(x, t) was
-      // issued (the S issuer waits for it)
-      const int pb = t & 1;
-      // 32 keys at a time: 16 packed FMAs, 32 ex2, four words of codes, one 16-byte store
-      uint8_t* p_row = s.p[x][pb] + r * kPRowBytes;
-      uint8_t* d_row = (DBG && dbg) ? p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) + t * kPRowBytes
-                                    : nullptr;
-      float tile_sum = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        float* y = sv + 32 * cc;
-        uint4 w4;
-        if constexpr (EFQ) {
-          // w = sat((2 r + 2) / 7); w times 7 * 2^-149 lands on the subnormal grid, so the product's
-          // bit pattern is round(7 w) in [0, 7] (round to nearest even): the code itself
-          const float b7 = fmaf(nb[cc], 2.f / 7.f, 2.f / 7.f);
-          uint32_t wd[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            float k[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) k[i] = fma_sat(y[8 * w + i], c27, b7);
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) fmul2_b(k[i], k[i + 1], k[i], k[i + 1], __uint_as_float(7u));
-            uint32_t acc = pack_u4x2(0u, __float_as_uint(k[7]), __float_as_uint(k[6]));
-            acc = pack_u4x2(acc, __float_as_uint(k[5]), __float_as_uint(k[4]));
-            acc = pack_u4x2(acc, __float_as_uint(k[3]), __float_as_uint(k[2]));
-            wd[w] = pack_u4x2(acc, __float_as_uint(k[1]), __float_as_uint(k[0]));
-          }
-          w4 = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float x0, x1;
-            ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
-            if (PM == 1 && poly_pair(i / 2)) {
-              exp2_codes_poly(y[i], y[i + 1], x0, x1);
-            } else {
-              y[i] = ex2_approx_ftz(x0);
-              y[i + 1] = ex2_approx_ftz(x1);
-            }
-          }
-          w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
-        }
-        *reinterpret_cast<uint4*>(p_row + ((cc ^ swz) << 4)) = w4;
-        if (DBG && dbg) reinterpret_cast<uint4*>(d_row)[cc] = w4;
-        if (!PNQ) {   // conventional row sum of the unquantized exponentials
-#pragma unroll
-          for (int bb = 0; bb < 32 / kPB; ++bb) {
-            float b0 = 0.f, b1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < kPB; i += 2) {
-              b0 += y[bb * kPB + i];
-              b1 += y[bb * kPB + i + 1];
-            }
-            tile_sum = fmaf(b0 + b1, bscale[(32 * cc) / kPB + bb], tile_sum);
-          }
-        }
-      }
-      if (!PNQ) l = fmaf(alpha, l, tile_sum);
-#pragma unroll
-      for (int a = 0; a < kNPB / 4; ++a) *reinterpret_cast<uint32_t*>(s.psf[x][pb] + a * 512 + psf_off) = sbytes[a];
-      if (DBG && dbg) {
-        uint32_t* ds = reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) *
-                                                                      (p.Npad / kPB) + t * kNPB);
-#pragma unroll
-        for (int a = 0; a < kNPB / 4; ++a) ds[a] = sbytes[a];
-      }
-      fence_proxy_async_smem();
-
-      // history rescale of O and L (only when some row of this warp saw its max move); O may only
-      // be touched once the product of key tile t-1 has landed in it
-      if (t > 0 && moved) {
-        ok = warp_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
+      for (int t = 0; ok && t < n_kv; ++t) {
+        ok = warp_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8);
         if (!ok) break;
         tc_fence_after();
+        float sv[kHalf];
         {
-          // O and (PNQ) L in one batch of loads behind one wait, then one batch of stores
-          uint32_t raw[D];
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc)
-            tmem_ld32(o_col + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
-          const uint32_t lv = PNQ ? tmem_ld1(l_col) : 0u;
+          uint32_t raw[kHalf];
+          tmem_ld16x2_64<kHalf>(tmem + lane_addr + kColS, raw);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < D; i += 2) {
-            float o0, o1;
-            fmul2_b(o0, o1, __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]), alpha);
-            raw[i] = __float_as_uint(o0);
-            raw[i + 1] = __float_as_uint(o1);
-          }
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc)
-            tmem_st32(o_col + cc * 32, *reinterpret_cast<const uint32_t(*)[32]>(raw + 32 * cc));
-          if (PNQ) tmem_st1(l_col, __float_as_uint(__uint_as_float(lv) * alpha));
+          for (int i = 0; i < kHalf; ++i) sv[i] = __uint_as_float(raw[i]);
         }
-        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bar_s_empty);
+
+        // masking: keys beyond N, and keys after the query row when causal
+        const int key0 = t * kBN + kh * kHalf;
+        if (t * kBN + kBN > p.N || (p.causal && t * kBN + kBN - 1 > qt * kBM)) {
+          const int lim = (p.causal ? min(p.N, qrow + 1) : p.N) - key0;   // keys [key0, key0 + lim) count
+#pragma unroll
+          for (int i = 0; i < kHalf; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
+        }
+        float bmax[kNPBt];
+#pragma unroll
+        for (int bb = 0; bb < kNPBt; ++bb) bmax[bb] = NV ? block_max16(sv + bb * kPB) : block_max32(sv + bb * kPB);
+        float tmax = bmax[0];
+#pragma unroll
+        for (int bb = 1; bb < kNPBt; ++bb) tmax = fmaxf(tmax, bmax[bb]);
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        const float m_new = fmaxf(m, tmax);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        // the history factor alpha = 2^((m - m') c) only where some row of the warp saw its max move
+        // (elsewhere it is 1); it is read by the rescale below and by the conventional row sum
+        const bool moved = __any_sync(0xffffffffu, m_new > m);
+        float alpha = 1.f;
+        if (moved) alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
+
+        uint32_t sbytes = 0;      // this thread's scale bytes, block order
+        float nb[kNPBt], bscale[kNPBt];
+#pragma unroll
+        for (int bb = 0; bb < kNPBt; ++bb) {
+          uint32_t byte;
+          if constexpr (NV) {
+            const float amax = ex2_approx((bmax[bb] - m_use) * c);   // 0 for an all-masked block
+            // s = E4M3(amax / 6), the quotient as amax times fp32(1/6): within one ulp of the
+            // correctly rounded quotient, so the E4M3 rounding can only differ where the quotient
+            // lies within an ulp of one of its midpoints (amax itself comes from ex2.approx). s = 0
+            // (amax <= 6 * 2^-10): y = P~ itself (every value below the 0.25 rounding threshold,
+            // so the codes are 0 as the format wants) and the unquantized row sum still counts the
+            // block with weight 1
+            byte = e4m3_byte(amax * (1.0f / 6.0f));
+            const float sb = e4m3_value(byte);
+            bscale[bb] = sb > 0.f ? sb : 1.f;
+            nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
+          } else {
+            // the byte of amax = 2^((bmax - m') c) straight from the exponent (no MUFU on this path)
+            byte = p_scale_byte_log2((bmax[bb] - m_use) * c, p.mode);
+            // 127 - byte as a float without a conversion: it sits in the low mantissa bits of 2^23
+            const float neg_e = __uint_as_float(0x4B000000u + (127u - byte)) - 8388608.0f;
+            nb[bb] = fmaf(-m_use, c, neg_e);
+            bscale[bb] = pow2_from_byte(byte);
+          }
+          sbytes |= byte << (8 * bb);
+        }
+        // P~ buffer t&1: its last reader, the product of key tile t-2, completed before S(x, t) was
+        // issued (the S issuer waits for it)
+        const int pb = t & 1;
+        // 32 keys at a time (this thread's two 16-byte pieces of the row)
+        uint8_t* p_row = s.p[x][pb] + r * kPRowBytes;
+        uint8_t* d_row = (DBG && dbg) ? p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) + t * kPRowBytes
+                                      : nullptr;
+        float tile_sum = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < kHalf / 32; ++cc) {
+          const int jc = kh * (kHalf / 32) + cc;          // 16-byte piece of the row
+          float* y = sv + 32 * cc;
+          uint4 w4;
+          if constexpr (EFQ) {
+            // w = sat((2 r + 2) / 7); w times 7 * 2^-149 lands on the subnormal grid, so the product's
+            // bit pattern is round(7 w) in [0, 7] (round to nearest even): the code itself
+            const float b7 = fmaf(nb[cc], 2.f / 7.f, 2.f / 7.f);
+            uint32_t wd[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              float k[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) k[i] = fma_sat(y[8 * w + i], c27, b7);
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) fmul2_b(k[i], k[i + 1], k[i], k[i + 1], __uint_as_float(7u));
+              uint32_t acc = pack_u4x2(0u, __float_as_uint(k[7]), __float_as_uint(k[6]));
+              acc = pack_u4x2(acc, __float_as_uint(k[5]), __float_as_uint(k[4]));
+              acc = pack_u4x2(acc, __float_as_uint(k[3]), __float_as_uint(k[2]));
+              wd[w] = pack_u4x2(acc, __float_as_uint(k[1]), __float_as_uint(k[0]));
+            }
+            w4 = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              float x0, x1;
+              ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
+              if (PM == 1 && poly_pair<kPolyPairs16>(i / 2)) {
+                exp2_codes_poly(y[i], y[i + 1], x0, x1);
+              } else {
+                y[i] = ex2_approx_ftz(x0);
+                y[i + 1] = ex2_approx_ftz(x1);
+              }
+            }
+            w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
+          }
+          *reinterpret_cast<uint4*>(p_row + ((static_cast<uint32_t>(jc) ^ swz) << 4)) = w4;
+          if (DBG && dbg) reinterpret_cast<uint4*>(d_row)[jc] = w4;
+          if (!PNQ) {   // conventional row sum of the unquantized exponentials
+#pragma unroll
+            for (int bb = 0; bb < 32 / kPB; ++bb) {
+              float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+              for (int i = 0; i < kPB; i += 2) {
+                b0 += y[bb * kPB + i];
+                b1 += y[bb * kPB + i + 1];
+              }
+              tile_sum = fmaf(b0 + b1, bscale[(32 * cc) / kPB + bb], tile_sum);
+            }
+          }
+        }
+        if (!PNQ) l = fmaf(alpha, l, tile_sum);
+        if constexpr (NV)   // two atoms per tile (keys 0-63, 64-127), four blocks each
+          *reinterpret_cast<uint32_t*>(s.psf[x][pb] + kh * 512 + psf_off) = sbytes;
+        else                // one atom, this thread's two of its four blocks
+          *reinterpret_cast<uint16_t*>(s.psf[x][pb] + psf_off + 2 * kh) = static_cast<uint16_t>(sbytes);
+        if (DBG && dbg) {
+          uint8_t* ds = p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / kPB) + t * kNPB + kh * kNPBt;
+#pragma unroll
+          for (int bb = 0; bb < kNPBt; ++bb) ds[bb] = static_cast<uint8_t>(sbytes >> (8 * bb));
+        }
+        fence_proxy_async_smem();
+
+        // history rescale of O and L (only when some row of this warp saw its max move); O may only
+        // be touched once the product of key tile t-1 has landed in it
+        if (t > 0 && moved) {
+          ok = warp_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
+          if (!ok) break;
+          tc_fence_after();
+          {
+            // this thread's half of O's columns, and L in the 16-lane x 2-column layout (thread t
+            // holds row (t >> 2) + 8 (t & 1) of the 16, whose alpha its row owner passes over)
+            uint32_t raw[D / 2];
+            tmem_ld16x2_h<D>(o_col, raw);
+            const uint32_t lv = PNQ ? tmem_ld16x64b_1(l_col) : 0u;
+            const float alpha_l = __shfl_sync(0xffffffffu, alpha, ((lane >> 2) + 8 * (lane & 1)));
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < D / 2; i += 2) {
+              float o0, o1;
+              fmul2_b(o0, o1, __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]), alpha);
+              raw[i] = __float_as_uint(o0);
+              raw[i + 1] = __float_as_uint(o1);
+            }
+            tmem_st16x2_h<D>(o_col, raw);
+            if (PNQ) tmem_st16x64b_1(l_col, __float_as_uint(__uint_as_float(lv) * alpha_l));
+          }
+          tc_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bar_p_full[x][pb]);
+        m = m_new;
+      }
+
+      // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
+      if (ok) {
+        ok = warp_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
+                       kStatusTimeoutPV | 1);
+      }
+      if (ok) {
+        tc_fence_after();
+        if (PNQ) {
+          uint32_t lv[1];
+          tmem_ld16x2_1<0>(l_col, lv);        // both halves read the row's sum in column 0
+          tc_wait_ld();
+          l = __uint_as_float(lv[0]);
+        } else {
+          l += __shfl_xor_sync(0xffffffffu, l, 16);
+        }
+        const float inv_l = 1.f / l;
+        // The normalised rows leave through shared memory so that the global writes are whole lines:
+        // per round, a 16-row x 128-byte stage (this warp's rows of the tile's two P~ buffers, which
+        // no product reads any more) takes the 128 bytes of each row that the round covers, written
+        // by the thread of the row that holds them, then the warp reads it back line-wise (eight
+        // lanes per line) and stores it. 128-byte swizzle: the 16-byte piece j of stage row rr sits
+        // at position j ^ (rr & 7). fp32: a round is 32 columns, bf16 64.
+        auto stage_row = [&](int rr) {
+          return smem_u32(s.p[x][rr >> 3]) + static_cast<uint32_t>(r0 + 2 * (rr & 7)) * kPRowBytes;
+        };
+        const int es = p.out_bf16 ? 2 : 4;
+        const int rounds = D * es / 128;
+        const int y0 = qt * kBM + r0;
+        uint8_t* const ohead = static_cast<uint8_t*>(p.out) + static_cast<size_t>(bh_q) * p.N * D * es;
+        const uint32_t my_row = stage_row(lane & 15);
+        const uint32_t rsw = static_cast<uint32_t>(lane) & 7u;
+#pragma unroll 1
+        for (int g = 0; g < rounds; ++g) {
+          if (p.out_bf16) {
+            // round g: columns [64 g, 64 g + 64); with D = 128 one half's whole range (half g),
+            // with D = 64 32 columns from each half
+            uint32_t ov[32];
+            tmem_ld16x2_32<D / 2>(o_col + (D == 128 ? 32u * 0u : 0u), ov);   // first 32 of each half
+            uint32_t ow[32];
+            tmem_ld16x2_32<D / 2>(o_col + (D == 128 ? 32u : 0u), ow);        // next 32 (D = 128)
+            tc_wait_ld();
+            const bool mine = (D == 128) ? (kh == g) : true;
+            if (mine) {
+#pragma unroll
+              for (int pc = 0; pc < (D == 128 ? 8 : 4); ++pc) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int i = 8 * pc + 2 * u;
+                  const float a0 = __uint_as_float(i < 32 ? ov[i & 31] : ow[i & 31]) * inv_l;
+                  const float a1 = __uint_as_float(i + 1 < 32 ? ov[(i + 1) & 31] : ow[(i + 1) & 31]) * inv_l;
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                  w[u] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                const int piece = (D == 128) ? pc : 4 * kh + pc;
+                st_shared_v4(my_row + ((static_cast<uint32_t>(piece) ^ rsw) << 4), w[0], w[1], w[2], w[3]);
+              }
+            }
+          } else {
+            // round g: columns [32 g, 32 g + 32), held by half g / (D / 64) at its offset 32 (g % (D / 64))
+            uint32_t ov[32];
+            tmem_ld16x2_32<D / 2>(o_col + 32u * static_cast<uint32_t>(g % (D / 64)), ov);
+            tc_wait_ld();
+            if (kh == g / (D / 64)) {
+#pragma unroll
+              for (int pc = 0; pc < 8; ++pc)
+                st_shared_v4(my_row + ((static_cast<uint32_t>(pc) ^ rsw) << 4),
+                             __float_as_uint(__uint_as_float(ov[4 * pc]) * inv_l),
+                             __float_as_uint(__uint_as_float(ov[4 * pc + 1]) * inv_l),
+                             __float_as_uint(__uint_as_float(ov[4 * pc + 2]) * inv_l),
+                             __float_as_uint(__uint_as_float(ov[4 * pc + 3]) * inv_l));
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int idx = it * 32 + lane;
+            const int rr = idx >> 3, pc = idx & 7;
+            const uint4 val = ld_shared_v4(stage_row(rr) + ((static_cast<uint32_t>(pc) ^ (static_cast<uint32_t>(rr) & 7u)) << 4));
+            if (y0 + rr < p.N)
+              *reinterpret_cast<uint4*>(ohead + static_cast<size_t>(y0 + rr) * D * es + g * 128 + pc * 16) = val;
+          }
+          __syncwarp();     // the stage is read before the next round overwrites it
+        }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.bar_p_full[x][pb]);
-      m = m_new;
-    }
+    } else {
 
-    // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
-    if (ok) {
-      ok = warp_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
-                     kStatusTimeoutPV | 1);
-    }
-    if (ok) {
-      tc_fence_after();
-      if (PNQ) {
-        l = __uint_as_float(tmem_ld1(l_col));
-        tc_wait_ld();
-      }
-      const float inv_l = 1.f / l;
-      // The normalised rows leave through shared memory so that the global writes are whole lines:
-      // each warp stages a 32-row x 128-byte chunk (32 fp32 or 64 bf16 columns, its threads' rows)
-      // in its quarter of its query tile's P~ buffers, which no product reads any more once the
-      // last P~V product has completed, then reads it back four rows per instruction (eight
-      // lanes per 128-byte line). 128-byte swizzle: the 16-byte piece j of row r sits at position
-      // j ^ (r & 7), so that neither the row-wise writes nor the line-wise reads conflict on banks.
-      uint8_t* stage = s.p[x][0] + quarter * 4096;
-      const uint32_t row_addr = smem_u32(stage) + static_cast<uint32_t>(lane) * 128u;
-      const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
-      const int y0 = qt * kBM + quarter * 32;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t raw[32];
-        tmem_ld32(o_col + cc * 32, raw);
-        tc_wait_ld();
-        const bool half2 = p.out_bf16 && (cc & 1);        // bf16: second half of a 128-byte row
-        if (p.out_bf16) {
+      // ============================ softmax warps ============================
+      const int x = (warp - 4) >> 2;                    // query tile: warps 4-7 A, 8-11 B
+      const int quarter = warp & 3;                     // TMEM lane quarter this warp may access
+      const int r = quarter * 32 + lane;                // row inside the tile == TMEM lane
+      const int qt = x == 0 ? qt_x[0] : qt_x[1];
+      const int n_kv = x == 0 ? n_kv_x[0] : n_kv_x[1];
+      const int qrow = qt * kBM + r;
+      const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t o_col = tmem + lane_addr + kColO + 128 * x;
+      const uint32_t l_col = tmem + lane_addr + kColL + 16 * x;
+      const float c = p.scale_log2;
+      constexpr int kPB = NV ? 16 : 32;                 // keys per P~ scale block
+      constexpr int kNPB = kBN / kPB;                   // scale blocks per row per tile
+      const float c27 = c * (2.f / 7.f);                // exp-free rule: (2 r + 2) / 7 = S c27 + b7
+      float m = -INFINITY;      // running max of the raw scores S
+      float l = 0.f;            // running row sum (pnq = 0)
+      bool ok = n_kv > 0;
+      const bool dbg = DBG && bh_q == p.dbg_bh && qrow >= p.dbg_r0 && qrow < p.dbg_r1;
+      const uint32_t swz = (static_cast<uint32_t>(r) >> 1) & 3u;   // 64-byte swizzle of this row
+      const uint32_t psf_off = (r & 31) * 16 + (r >> 5) * 4;
+
+      for (int t = 0; ok && t < n_kv; ++t) {
+        ok = warp_wait(&s.bar_s_full[x], t & 1, abort_flag, p.status, kStatusTimeoutS | 8);
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kBN];
+        {
+          uint32_t raw[kBN];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t wv[4];
+          for (int cc = 0; cc < kBN / 32; ++cc)
+            tmem_ld32(tmem + lane_addr + kColS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
+          tc_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * u]) * inv_l,
-                                                              __uint_as_float(raw[v * 8 + 2 * u + 1]) * inv_l);
-              wv[u] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(raw[i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bar_s_empty);
+
+        // masking: keys beyond N, and keys after the query row when causal
+        const int key0 = t * kBN;
+        if (key0 + kBN > p.N || (p.causal && key0 + kBN - 1 > qt * kBM)) {
+          const int lim = (p.causal ? min(p.N, qrow + 1) : p.N) - key0;   // keys [key0, key0 + lim) count
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
+        }
+        // per block (32 keys for MXFP4, 16 for NVFP4): amax from the exact difference (1 for the
+        // block that holds the max), the block's scale byte, and the exponent bias nb of
+        // y = P~ / s = 2^(S c - m c - log2 s): one packed FMA per two elements and one ex2 each
+        float bmax[kNPB];
+#pragma unroll
+        for (int bb = 0; bb < kNPB; ++bb) bmax[bb] = NV ? block_max16(sv + bb * kPB) : block_max32(sv + bb * kPB);
+        float tmax = bmax[0];
+#pragma unroll
+        for (int bb = 1; bb < kNPB; ++bb) tmax = fmaxf(tmax, bmax[bb]);
+        const float m_new = fmaxf(m, tmax);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        // the history factor alpha = 2^((m - m') c) only where some row of the warp saw its max move
+        // (elsewhere it is 1); it is read by the rescale below and by the conventional row sum
+        const bool moved = __any_sync(0xffffffffu, m_new > m);
+        float alpha = 1.f;
+        if (moved) alpha = (m == -INFINITY) ? 0.f : ex2_approx((m - m_use) * c);
+
+        uint32_t sbytes[kNPB / 4];
+        float nb[kNPB], bscale[kNPB];
+#pragma unroll
+        for (int bb = 0; bb < kNPB; ++bb) {
+          uint32_t byte;
+          if constexpr (NV) {
+            const float amax = ex2_approx((bmax[bb] - m_use) * c);   // 0 for an all-masked block
+            // s = E4M3(amax / 6), the quotient as amax times fp32(1/6): within one ulp of the
+            // correctly rounded quotient, so the E4M3 rounding can only differ where the quotient
+            // lies within an ulp of one of its midpoints (amax itself comes from ex2.approx). s = 0
+            // (amax <= 6 * 2^-10): y = P~ itself (every value below the 0.25 rounding threshold,
+            // so the codes are 0 as the format wants) and the unquantized row sum still counts the
+            // block with weight 1
+            byte = e4m3_byte(amax * (1.0f / 6.0f));
+            const float sb = e4m3_value(byte);
+            bscale[bb] = sb > 0.f ? sb : 1.f;
+            nb[bb] = sb > 0.f ? fmaf(-m_use, c, -lg2_approx(sb)) : -m_use * c;
+          } else {
+            // the byte of amax = 2^((bmax - m') c) straight from the exponent (no MUFU on this path)
+            byte = p_scale_byte_log2((bmax[bb] - m_use) * c, p.mode);
+            // 127 - byte as a float without a conversion: it sits in the low mantissa bits of 2^23
+            const float neg_e = __uint_as_float(0x4B000000u + (127u - byte)) - 8388608.0f;
+            nb[bb] = fmaf(-m_use, c, neg_e);
+            bscale[bb] = pow2_from_byte(byte);
+          }
+          if (bb % 4 == 0) sbytes[bb / 4] = 0;
+          sbytes[bb / 4] |= byte << (8 * (bb % 4));
+        }
+        // P~ buffer t&1: its last reader, the product of key tile t-2, completed before S(x, t) was
+        // issued (the S issuer waits for it)
+        const int pb = t & 1;
+        // 32 keys at a time: 16 packed FMAs, 32 ex2, four words of codes, one 16-byte store
+        uint8_t* p_row = s.p[x][pb] + r * kPRowBytes;
+        uint8_t* d_row = (DBG && dbg) ? p.dbg_codes + static_cast<size_t>(qrow - p.dbg_r0) * (p.Npad / 2) + t * kPRowBytes
+                                      : nullptr;
+        float tile_sum = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          float* y = sv + 32 * cc;
+          uint4 w4;
+          if constexpr (EFQ) {
+            // w = sat((2 r + 2) / 7); w times 7 * 2^-149 lands on the subnormal grid, so the product's
+            // bit pattern is round(7 w) in [0, 7] (round to nearest even): the code itself
+            const float b7 = fmaf(nb[cc], 2.f / 7.f, 2.f / 7.f);
+            uint32_t wd[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              float k[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) k[i] = fma_sat(y[8 * w + i], c27, b7);
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) fmul2_b(k[i], k[i + 1], k[i], k[i + 1], __uint_as_float(7u));
+              uint32_t acc = pack_u4x2(0u, __float_as_uint(k[7]), __float_as_uint(k[6]));
+              acc = pack_u4x2(acc, __float_as_uint(k[5]), __float_as_uint(k[4]));
+              acc = pack_u4x2(acc, __float_as_uint(k[3]), __float_as_uint(k[2]));
+              wd[w] = pack_u4x2(acc, __float_as_uint(k[1]), __float_as_uint(k[0]));
             }
-            st_shared_v4(row_addr + ((((half2 ? 4u : 0u) + v) ^ sw) << 4), wv[0], wv[1], wv[2], wv[3]);
-          }
-        } else {
+            w4 = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          } else {
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            st_shared_v4(row_addr + ((static_cast<uint32_t>(v) ^ sw) << 4),
-                         __float_as_uint(__uint_as_float(raw[4 * v]) * inv_l),
-                         __float_as_uint(__uint_as_float(raw[4 * v + 1]) * inv_l),
-                         __float_as_uint(__uint_as_float(raw[4 * v + 2]) * inv_l),
-                         __float_as_uint(__uint_as_float(raw[4 * v + 3]) * inv_l));
+            for (int i = 0; i < 32; i += 2) {
+              float x0, x1;
+              ffma2_bc(x0, x1, y[i], y[i + 1], c, nb[(32 * cc + i) / kPB]);
+              if (PM == 1 && poly_pair<kPolyPairs8>(i / 2)) {
+                exp2_codes_poly(y[i], y[i + 1], x0, x1);
+              } else {
+                y[i] = ex2_approx_ftz(x0);
+                y[i + 1] = ex2_approx_ftz(x1);
+              }
+            }
+            w4 = make_uint4(cvt_e2m1x8(y), cvt_e2m1x8(y + 8), cvt_e2m1x8(y + 16), cvt_e2m1x8(y + 24));
+          }
+          *reinterpret_cast<uint4*>(p_row + ((cc ^ swz) << 4)) = w4;
+          if (DBG && dbg) reinterpret_cast<uint4*>(d_row)[cc] = w4;
+          if (!PNQ) {   // conventional row sum of the unquantized exponentials
+#pragma unroll
+            for (int bb = 0; bb < 32 / kPB; ++bb) {
+              float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+              for (int i = 0; i < kPB; i += 2) {
+                b0 += y[bb * kPB + i];
+                b1 += y[bb * kPB + i + 1];
+              }
+              tile_sum = fmaf(b0 + b1, bscale[(32 * cc) / kPB + bb], tile_sum);
+            }
+          }
         }
-        if (!p.out_bf16 || half2) {
-          __syncwarp();
-          const int es = p.out_bf16 ? 2 : 4;
-          const int pc = lane & 7;
-          uint8_t* gbase = static_cast<uint8_t*>(p.out) + static_cast<size_t>(bh_q) * p.N * D * es +
-                           (p.out_bf16 ? (cc >> 1) * 128 : cc * 128) + pc * 16;
+        if (!PNQ) l = fmaf(alpha, l, tile_sum);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int rr = 4 * k + (lane >> 3);
-            const uint4 val = ld_shared_v4(smem_u32(stage) + rr * 128 + ((pc ^ (rr & 7)) << 4));
-            if (y0 + rr < p.N) *reinterpret_cast<uint4*>(gbase + static_cast<size_t>(y0 + rr) * D * es) = val;
+        for (int a = 0; a < kNPB / 4; ++a) *reinterpret_cast<uint32_t*>(s.psf[x][pb] + a * 512 + psf_off) = sbytes[a];
+        if (DBG && dbg) {
+          uint32_t* ds = reinterpret_cast<uint32_t*>(p.dbg_scales + static_cast<size_t>(qrow - p.dbg_r0) *
+                                                                        (p.Npad / kPB) + t * kNPB);
+#pragma unroll
+          for (int a = 0; a < kNPB / 4; ++a) ds[a] = sbytes[a];
+        }
+        fence_proxy_async_smem();
+
+        // history rescale of O and L (only when some row of this warp saw its max move); O may only
+        // be touched once the product of key tile t-1 has landed in it
+        if (t > 0 && moved) {
+          ok = warp_wait(&s.bar_pv_done[x][pb ^ 1], ((t - 1) >> 1) & 1, abort_flag, p.status, kStatusTimeoutPV | 4);
+          if (!ok) break;
+          tc_fence_after();
+          {
+            // O and (PNQ) L in one batch of loads behind one wait, then one batch of stores
+            uint32_t raw[D];
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc)
+              tmem_ld32(o_col + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32 * cc));
+            const uint32_t lv = PNQ ? tmem_ld1(l_col) : 0u;
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < D; i += 2) {
+              float o0, o1;
+              fmul2_b(o0, o1, __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]), alpha);
+              raw[i] = __float_as_uint(o0);
+              raw[i + 1] = __float_as_uint(o1);
+            }
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc)
+              tmem_st32(o_col + cc * 32, *reinterpret_cast<const uint32_t(*)[32]>(raw + 32 * cc));
+            if (PNQ) tmem_st1(l_col, __float_as_uint(__uint_as_float(lv) * alpha));
           }
-          __syncwarp();     // the stage is read before the next chunk overwrites it
+          tc_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bar_p_full[x][pb]);
+        m = m_new;
+      }
+
+      // ---- epilogue: out = O / l (PV products complete in order: the last one covers all)
+      if (ok) {
+        ok = warp_wait(&s.bar_pv_done[x][(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, p.status,
+                       kStatusTimeoutPV | 1);
+      }
+      if (ok) {
+        tc_fence_after();
+        if (PNQ) {
+          l = __uint_as_float(tmem_ld1(l_col));
+          tc_wait_ld();
+        }
+        const float inv_l = 1.f / l;
+        // The normalised rows leave through shared memory so that the global writes are whole lines:
+        // each warp stages a 32-row x 128-byte chunk (32 fp32 or 64 bf16 columns, its threads' rows)
+        // in its quarter of its query tile's P~ buffers, which no product reads any more once the
+        // last P~V product has completed, then reads it back four rows per instruction (eight
+        // lanes per 128-byte line). 128-byte swizzle: the 16-byte piece j of row r sits at position
+        // j ^ (r & 7), so that neither the row-wise writes nor the line-wise reads conflict on banks.
+        uint8_t* stage = s.p[x][0] + quarter * 4096;
+        const uint32_t row_addr = smem_u32(stage) + static_cast<uint32_t>(lane) * 128u;
+        const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
+        const int y0 = qt * kBM + quarter * 32;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t raw[32];
+          tmem_ld32(o_col + cc * 32, raw);
+          tc_wait_ld();
+          const bool half2 = p.out_bf16 && (cc & 1);        // bf16: second half of a 128-byte row
+          if (p.out_bf16) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(raw[v * 8 + 2 * u]) * inv_l,
+                                                                __uint_as_float(raw[v * 8 + 2 * u + 1]) * inv_l);
+                wv[u] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+              st_shared_v4(row_addr + ((((half2 ? 4u : 0u) + v) ^ sw) << 4), wv[0], wv[1], wv[2], wv[3]);
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              st_shared_v4(row_addr + ((static_cast<uint32_t>(v) ^ sw) << 4),
+                           __float_as_uint(__uint_as_float(raw[4 * v]) * inv_l),
+                           __float_as_uint(__uint_as_float(raw[4 * v + 1]) * inv_l),
+                           __float_as_uint(__uint_as_float(raw[4 * v + 2]) * inv_l),
+                           __float_as_uint(__uint_as_float(raw[4 * v + 3]) * inv_l));
+          }
+          if (!p.out_bf16 || half2) {
+            __syncwarp();
+            const int es = p.out_bf16 ? 2 : 4;
+            const int pc = lane & 7;
+            uint8_t* gbase = static_cast<uint8_t*>(p.out) + static_cast<size_t>(bh_q) * p.N * D * es +
+                             (p.out_bf16 ? (cc >> 1) * 128 : cc * 128) + pc * 16;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int rr = 4 * k + (lane >> 3);
+              const uint4 val = ld_shared_v4(smem_u32(stage) + rr * 128 + ((pc ^ (rr & 7)) << 4));
+              if (y0 + rr < p.N) *reinterpret_cast<uint4*>(gbase + static_cast<size_t>(y0 + rr) * D * es) = val;
+            }
+            __syncwarp();     // the stage is read before the next chunk overwrites it
+          }
         }
       }
+      tc_fence_before();
     }
-    tc_fence_before();
   }
 
   __syncthreads();
@@ -809,7 +1130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int PM, bool DBG, bool NV>
+template <int D, int PM, bool DBG, bool NV, int WS>
 static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D>();
@@ -818,18 +1139,29 @@ static cudaError_t launch_k(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
-    cudaError_t ea = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, PM, DBG, NV>);
+    cudaError_t ea = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, PM, DBG, NV, WS>);
     if (ea != cudaSuccess) return ea;
     regs = fa.numRegs;
   }
-  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PM, DBG, NV>,
+  if (regs != Layout<WS>::kLaunchRegs) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, PM, DBG, NV, WS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned n_units = static_cast<unsigned>((p.Npad / kBM + 1) / 2);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * n_units;
-  mxattn_fwd_kernel<D, PM, DBG, NV><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
+  mxattn_fwd_kernel<D, PM, DBG, NV, WS><<<grid, Layout<WS>::kThreads, smem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
+}
+
+// Softmax layout per launch (measured on the benchmark workloads): two threads per row for
+// exp-then-quantize without a causal mask (video-DiT PNQ +2%, NVFP4 +2%, pnq = 0 +1%); one thread
+// per row for the exp-free rule (the two-thread layout is 8% slower there) and for causal
+// attention (1% slower there: more of its time is per-unit work).
+template <int D, int PM, bool DBG, bool NV>
+static cudaError_t launch_w(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const AttnParams& p, cudaStream_t stream) {
+  if (PM != 2 && !p.causal) return launch_k<D, PM, DBG, NV, 8>(tmQ, tmK, tmV, p, stream);
+  return launch_k<D, PM, DBG, NV, 4>(tmQ, tmK, tmV, p, stream);
 }
 
 template <int D, bool NV>
@@ -838,13 +1170,13 @@ static cudaError_t launch_f(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
   const bool dbg = p.dbg_codes != nullptr;
   if (p.pnq == 2) {
     if constexpr (NV) return cudaErrorInvalidValue;    // the exp-free rule is MXFP4 only
-    else return dbg ? launch_k<D, 2, true, NV>(tmQ, tmK, tmV, p, stream)
-                    : launch_k<D, 2, false, NV>(tmQ, tmK, tmV, p, stream);
+    else return dbg ? launch_w<D, 2, true, NV>(tmQ, tmK, tmV, p, stream)
+                    : launch_w<D, 2, false, NV>(tmQ, tmK, tmV, p, stream);
   }
-  if (p.pnq == 1) return dbg ? launch_k<D, 1, true, NV>(tmQ, tmK, tmV, p, stream)
-                             : launch_k<D, 1, false, NV>(tmQ, tmK, tmV, p, stream);
-  return dbg ? launch_k<D, 0, true, NV>(tmQ, tmK, tmV, p, stream)
-             : launch_k<D, 0, false, NV>(tmQ, tmK, tmV, p, stream);
+  if (p.pnq == 1) return dbg ? launch_w<D, 1, true, NV>(tmQ, tmK, tmV, p, stream)
+                             : launch_w<D, 1, false, NV>(tmQ, tmK, tmV, p, stream);
+  return dbg ? launch_w<D, 0, true, NV>(tmQ, tmK, tmV, p, stream)
+             : launch_w<D, 0, false, NV>(tmQ, tmK, tmV, p, stream);
 }
 
 template <int D>
