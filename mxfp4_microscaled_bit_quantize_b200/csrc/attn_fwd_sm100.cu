@@ -21,8 +21,8 @@
 // S(A, t+1), ... . Their softmax warps therefore run half a step apart, and on every SM
 // sub-partition one tile's serial work (S load, maxima, scale selection, stores, rescale) overlaps
 // the other tile's exponentials on the MUFU.
-// Warp roles (384 threads, three warpgroups; setmaxnreg gives the control warpgroup 88 registers
-// per thread and each softmax warpgroup 208):
+// Warp roles (control warpgroup 0, then the softmax warpgroups; the layout WS is chosen per
+// launch, see Layout and launch_w):
 //   warp 2     TMA producer: Q tiles A and B once, then K / V^T tiles and their scale atoms into
 //              an NSTAGE-deep shared-memory ring (mbarrier complete_tx).
 //   warp 1     TMEM owner and S issuer (one thread): copies the Q and K scale atoms and issues
@@ -32,12 +32,16 @@
 //              TMEM and issue O_X += P~_X(t) V(t) and L_X += P~_X(t) 1 as soon as tile X's softmax
 //              hands P~ over. The four control warps sit on the four SM sub-partitions, so that the
 //              tcgen05 issue work is spread next to all eight softmax warps, which set the pace.
-//   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per query row (TMEM lane = row).
-//              Per key tile a thread reads its 128 scores with tcgen05.ld, releases S, updates the
-//              running max, computes P~ / 2^e per 32-key block, quantizes it in registers, writes
-//              64 bytes of codes (64B-swizzled, the MMA operand layout) and four scale bytes to
-//              shared memory, rescales O and L in TMEM when the max moves, and at the end
-//              normalises and stores the output row.
+//   WS = 4     warps 4-7 softmax of tile A, warps 8-11 of tile B (384 threads): one thread per
+//              query row (TMEM lane = row). Per key tile a thread reads its 128 scores with
+//              tcgen05.ld, releases S, updates the running max, computes P~ / 2^e per 32-key
+//              block, quantizes it in registers, writes 64 bytes of codes (64B-swizzled, the MMA
+//              operand layout) and four scale bytes to shared memory, rescales O and L in TMEM
+//              when the max moves, and at the end normalises and stores the output row.
+//   WS = 8     warps 4-11 tile A, 12-19 tile B (640 threads): two threads per query row, each
+//              with one 64-key half of every key tile (a 16-lane, two-half tcgen05.ld), so that
+//              each SM sub-partition runs four softmax warps; the row max and the conventional
+//              row sum meet over one shuffle, everything else is per thread as above.
 // TMEM (512 columns): S [0,128) O_A [128,128+d) O_B [256,256+d) L_A [384,400) L_B [400,416),
 // scale atoms from 416 (see kColSf*).
 // The kernel is templated on the format: MXFP4 (the method) or, for comparison, NVFP4 (blocks of
