@@ -71,7 +71,7 @@ def profile_traffic(name: str, src_hash: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms during the timed region. The
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms during the timed region. The
     sampler starts first; entering returns once its first sample has arrived (or after 3 s), and
     only the samples that arrive between entry and exit are summarised (all of them if none do)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -94,7 +94,7 @@ class ClockSampler:
         import shutil
         import threading
         cmd = ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "100"]
+               "-lms", "50"]
         if shutil.which("stdbuf"):
             cmd = ["stdbuf", "-oL"] + cmd      # one line per sample as it is taken
         try:
@@ -657,7 +657,7 @@ def run_quantizer_only(args, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=4096)
