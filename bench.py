@@ -245,7 +245,9 @@ def run_reference(args, rank: int) -> None:
     if rank != 0:
         return
     cfg = synthetic.ATTN_CONFIGS[WORKLOAD]
-    rows = args.ref_rows
+    # query rows per step: 10240 over the timed steps (512 a step at 20 steps, at least 128), so
+    # that more steps take fewer rows each; each step also quantizes the head's Q/K/V (a fixed cost)
+    rows = args.ref_rows if args.ref_rows else max(128, min(512, 10240 // max(1, args.steps)))
     for _ in range(args.warmup):
         oracle_sample(cfg, rows)
     flops = secs = 0.0
@@ -661,7 +663,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=4096)
-    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=0, help="query rows per reference step (0: 10240 / steps, 128..512)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", choices=["full", "attention", "quantizer", "gemm"], default="full",
                     help="attention / quantizer: time only that part (small cases for profiling)")
